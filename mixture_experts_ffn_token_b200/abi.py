@@ -1,0 +1,191 @@
+"""ctypes binding of the C ABI in include/moe.h.
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels
+of libmoe_b200.so.  Tensors are torch tensors already on the device; their
+data pointers and the current CUDA stream are passed through unchanged.
+There is no fallback: if the library is missing, loading it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
+
+MOE_OK = 0
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARGUMENT", 2: "MOE_ERR_UNSUPPORTED",
+                3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT"}
+ROUTERS = {"softmax_topk": 0, "sigmoid_sink": 1}
+FORMATS = {"concatenated": 0, "interleaved": 1}
+ACTIVATIONS = {"silu": 0, "swigluoai": 1, "gelu_tanh": 2}
+DTYPES = {torch.bfloat16: 0, torch.float32: 1}
+DEVICE_ERR_EXPERT_INDEX = 0x1
+DEVICE_ERR_CSR = 0x2
+DEVICE_ERR_TIMEOUT_GEMM1 = 0x4
+DEVICE_ERR_TIMEOUT_GEMM2 = 0x8
+NUM_STAGE_EVENTS = 9
+STAGE_NAMES = ("router", "csr_count", "csr_scan", "csr_scatter", "gather", "gemm_gate_up", "gemm_down", "combine")
+
+EXPORTED = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_create_indices", "moe_grouped_ffn",
+            "moe_forward", "moe_forward_timed", "moe_device_status")
+
+
+class MoEConfig(ctypes.Structure):
+    """moe_config_t."""
+    _fields_ = [
+        ("num_tokens", ctypes.c_int32),
+        ("hidden_dim", ctypes.c_int32),
+        ("num_experts", ctypes.c_int32),
+        ("top_k", ctypes.c_int32),
+        ("moe_dim", ctypes.c_int32),
+        ("num_sink", ctypes.c_int32),
+        ("router", ctypes.c_int),
+        ("logits_dtype", ctypes.c_int),
+        ("logits_row_stride", ctypes.c_int64),
+        ("route_scale", ctypes.c_float),
+        ("gate_up_format", ctypes.c_int),
+        ("activation", ctypes.c_int),
+        ("alpha", ctypes.c_float),
+        ("limit", ctypes.c_float),
+        ("has_bias", ctypes.c_int32),
+    ]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+_lib = None
+
+
+def load_library():
+    """Load libmoe_b200.so (raises OSError when it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise OSError(f"{LIB_PATH} is missing: build it with `python -m mixture_experts_ffn_token_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, cfgp, sz = ctypes.c_void_p, ctypes.POINTER(MoEConfig), ctypes.c_size_t
+    lib.moe_status_string.restype = ctypes.c_char_p
+    lib.moe_status_string.argtypes = [ctypes.c_int]
+    lib.moe_workspace_size.restype = ctypes.c_int
+    lib.moe_workspace_size.argtypes = [cfgp, ctypes.POINTER(ctypes.c_size_t)]
+    lib.moe_route.restype = ctypes.c_int
+    lib.moe_route.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp]
+    lib.moe_create_indices.restype = ctypes.c_int
+    lib.moe_create_indices.argtypes = [cfgp, vp, vp, vp, vp, vp, sz, vp]
+    lib.moe_grouped_ffn.restype = ctypes.c_int
+    lib.moe_grouped_ffn.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.moe_forward.restype = ctypes.c_int
+    lib.moe_forward.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.moe_forward_timed.restype = ctypes.c_int
+    lib.moe_forward_timed.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+    lib.moe_device_status.restype = ctypes.c_int
+    lib.moe_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
+    _lib = lib
+    return lib
+
+
+def make_config(wl, num_tokens: Optional[int] = None, logits_dtype=torch.float32,
+                logits_row_stride: Optional[int] = None) -> MoEConfig:
+    """moe_config_t for a workloads.Workload (num_tokens overrides wl's T)."""
+    c = MoEConfig()
+    c.num_tokens = wl.num_tokens if num_tokens is None else num_tokens
+    c.hidden_dim = wl.hidden_dim
+    c.num_experts = wl.num_experts
+    c.top_k = wl.top_k
+    c.moe_dim = wl.moe_dim
+    c.num_sink = wl.num_sink
+    c.router = ROUTERS[wl.router]
+    c.logits_dtype = DTYPES[logits_dtype]
+    c.logits_row_stride = wl.num_experts + wl.num_sink if logits_row_stride is None else logits_row_stride
+    c.route_scale = wl.route_scale
+    c.gate_up_format = FORMATS[wl.gate_up_format]
+    c.activation = ACTIVATIONS[wl.activation]
+    c.alpha = wl.alpha
+    c.limit = wl.limit
+    c.has_bias = 1 if wl.has_bias else 0
+    return c
+
+
+def _p(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoEError(status, where)
+
+
+def moe_status_string(status: int) -> str:
+    return load_library().moe_status_string(status).decode()
+
+
+def moe_workspace_size(cfg: MoEConfig) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().moe_workspace_size(ctypes.byref(cfg), ctypes.byref(n)), "moe_workspace_size")
+    return n.value
+
+
+def moe_route(cfg, logits, expert_indices, expert_weights, sink_weights=None, expert_bias=None,
+              global_scale=None, stream=None):
+    _check(load_library().moe_route(ctypes.byref(cfg), _p(logits), _p(expert_bias), _p(global_scale),
+                                    _p(expert_indices), _p(expert_weights), _p(sink_weights), _stream(stream)),
+           "moe_route")
+
+
+def moe_create_indices(cfg, expert_indices, expert_offsets, permutation, inverse, workspace, stream=None):
+    _check(load_library().moe_create_indices(ctypes.byref(cfg), _p(expert_indices), _p(expert_offsets),
+                                             _p(permutation), _p(inverse), _p(workspace), workspace.numel(),
+                                             _stream(stream)), "moe_create_indices")
+
+
+def moe_grouped_ffn(cfg, x, gate_up_w, gate_up_b, down_w, down_b, expert_offsets, permutation, expert_weights,
+                    out, workspace, stream=None):
+    _check(load_library().moe_grouped_ffn(ctypes.byref(cfg), _p(x), _p(gate_up_w), _p(gate_up_b), _p(down_w),
+                                          _p(down_b), _p(expert_offsets), _p(permutation), _p(expert_weights),
+                                          _p(out), _p(workspace), workspace.numel(), _stream(stream)),
+           "moe_grouped_ffn")
+
+
+def moe_forward(cfg, x, logits, gate_up_w, down_w, out, workspace, gate_up_b=None, down_b=None, expert_bias=None,
+                global_scale=None, expert_indices_out=None, expert_weights_out=None, sink_weights_out=None,
+                stream=None):
+    _check(load_library().moe_forward(ctypes.byref(cfg), _p(x), _p(logits), _p(expert_bias), _p(global_scale),
+                                      _p(gate_up_w), _p(gate_up_b), _p(down_w), _p(down_b), _p(out),
+                                      _p(expert_indices_out), _p(expert_weights_out), _p(sink_weights_out),
+                                      _p(workspace), workspace.numel(), _stream(stream)), "moe_forward")
+
+
+def moe_forward_timed(cfg, events, x, logits, gate_up_w, down_w, out, workspace, gate_up_b=None, down_b=None,
+                      expert_bias=None, global_scale=None, expert_indices_out=None, expert_weights_out=None,
+                      sink_weights_out=None, stream=None):
+    """moe_forward recording torch.cuda.Event objects `events` (9) between stages."""
+    arr = (ctypes.c_void_p * NUM_STAGE_EVENTS)(*[ev.cuda_event for ev in events])
+    _check(load_library().moe_forward_timed(ctypes.byref(cfg), _p(x), _p(logits), _p(expert_bias),
+                                            _p(global_scale), _p(gate_up_w), _p(gate_up_b), _p(down_w), _p(down_b),
+                                            _p(out), _p(expert_indices_out), _p(expert_weights_out),
+                                            _p(sink_weights_out), _p(workspace), workspace.numel(),
+                                            _stream(stream), arr), "moe_forward_timed")
+
+
+def moe_device_status(workspace, stream=None) -> int:
+    """The device fault bits recorded in the workspace (synchronizes the stream)."""
+    v = ctypes.c_int32(0)
+    st = load_library().moe_device_status(_p(workspace), ctypes.byref(v), _stream(stream))
+    if st not in (MOE_OK, 5):
+        raise MoEError(st, "moe_device_status")
+    return v.value

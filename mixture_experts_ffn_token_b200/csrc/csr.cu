@@ -1,0 +1,240 @@
+// csr.cu -- stage 2 (moe_create_indices) plus the two bandwidth kernels
+// around the grouped GEMMs (row gather and the k-way combine).
+//
+// moe_create_indices is named on the Mojo sink_gate_router_kernel page as the
+// separate bucketing step (it needs every token's assignment, a grid-wide
+// dependency); its outputs follow NeMo _permute_tokens_for_grouped_mm: the
+// routed slots sorted by expert, the per-expert counts and their cumulative
+// offsets.  Here the sort is a stable counting sort in three kernels:
+//   count   each CTA histograms one chunk of 2048 slots in shared memory;
+//   scan    one CTA turns the chunk histograms into per-expert offsets and
+//           per-(chunk, expert) base positions;
+//   scatter each CTA walks its chunk in slot order: every warp owns 128
+//           consecutive slots, __match_any_sync groups equal experts inside a
+//           32-slot step, a per-warp count table (scanned across warps) gives
+//           the position of each slot, so the order inside an expert is the
+//           slot order and no atomic decides any position.
+#include "kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kCsrWarps = kCsrThreads / 32;
+constexpr int kSlotsPerWarp = kCsrChunk / kCsrWarps;  // 128
+static_assert(kSlotsPerWarp % 32 == 0, "slots per warp must be whole warp steps");
+
+__global__ void __launch_bounds__(kCsrThreads) csr_count_kernel(const int32_t* __restrict__ idx, int R, int E,
+                                                                int32_t* __restrict__ chunk_counts, int* status) {
+  extern __shared__ int cnt[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kCsrChunk;
+  const int64_t end = min(base + kCsrChunk, static_cast<int64_t>(R));
+  bool bad = false;
+  for (int64_t s = base + threadIdx.x; s < end; s += blockDim.x) {
+    const int e = idx[s];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+    else bad = true;
+  }
+  if (bad) atomicOr(status, MOE_DEVICE_ERR_EXPERT_INDEX);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[static_cast<int64_t>(blockIdx.x) * E + e] = cnt[e];
+}
+
+// One CTA of 1024 threads; thread e owns expert e (E <= 1024).
+__global__ void __launch_bounds__(1024) csr_scan_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int E,
+                                                        int32_t* __restrict__ chunk_base,
+                                                        int32_t* __restrict__ offsets) {
+  __shared__ int warp_tot[32];
+  const int e = threadIdx.x;
+  const int lane = e & 31, warp = e >> 5;
+  int total = 0;
+  if (e < E) {
+    for (int c = 0; c < nchunks; ++c) {
+      const int64_t i = static_cast<int64_t>(c) * E + e;
+      const int v = chunk_counts[i];
+      chunk_base[i] = total;
+      total += v;
+    }
+  }
+  // exclusive scan of `total` over experts
+  int incl = total;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = warp_tot[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += y;
+    }
+    warp_tot[lane] = v;  // inclusive prefix of warp totals
+  }
+  __syncthreads();
+  const int excl = incl - total + (warp > 0 ? warp_tot[warp - 1] : 0);
+  if (e < E) {
+    offsets[e] = excl;
+    for (int c = 0; c < nchunks; ++c) chunk_base[static_cast<int64_t>(c) * E + e] += excl;
+  }
+  if (e == E - 1) offsets[E] = excl + total;
+}
+
+__global__ void __launch_bounds__(kCsrThreads) csr_scatter_kernel(const int32_t* __restrict__ idx, int R, int E,
+                                                                  const int32_t* __restrict__ chunk_base,
+                                                                  int32_t* __restrict__ perm,
+                                                                  int32_t* __restrict__ inv) {
+  extern __shared__ int wcnt[];  // [kCsrWarps][E]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kCsrWarps * E; i += blockDim.x) wcnt[i] = 0;
+  __syncthreads();
+  const int64_t wbase = static_cast<int64_t>(blockIdx.x) * kCsrChunk + static_cast<int64_t>(warp) * kSlotsPerWarp;
+  int* my = wcnt + warp * E;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  // pass 1: per-warp histogram
+  for (int r = 0; r < kSlotsPerWarp; r += 32) {
+    const int64_t s = wbase + r + lane;
+    const int e = s < R ? idx[s] : -1;
+    const bool ok = e >= 0 && e < E;
+    const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : E + lane);
+    if (ok && (peers & lt_mask) == 0) my[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // exclusive scan over warps, per expert
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < kCsrWarps; ++w) {
+      const int v = wcnt[w * E + e];
+      wcnt[w * E + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  // pass 2: positions in slot order
+  const int32_t* cb = chunk_base + static_cast<int64_t>(blockIdx.x) * E;
+  for (int r = 0; r < kSlotsPerWarp; r += 32) {
+    const int64_t s = wbase + r + lane;
+    const int e = s < R ? idx[s] : -1;
+    const bool ok = e >= 0 && e < E;
+    const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : E + lane);
+    int base = 0;
+    if (ok) base = cb[e] + my[e];
+    __syncwarp();
+    if (ok) {
+      const int pos = base + __popc(peers & lt_mask);
+      perm[pos] = static_cast<int32_t>(s);
+      if (inv != nullptr) inv[s] = pos;
+      if ((peers & lt_mask) == 0) my[e] += __popc(peers);
+    }
+    __syncwarp();
+  }
+}
+
+// One warp per gathered row: Xp[p, :] = x[perm[p] / k, :], 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          const int32_t* __restrict__ perm,
+                                                          const int32_t* __restrict__ offsets, int E, int R, int k,
+                                                          int H, __nv_bfloat16* __restrict__ Xp, int* status) {
+  int total = offsets[E];
+  if (total < 0 || total > R) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, MOE_DEVICE_ERR_CSR);
+    total = total < 0 ? 0 : R;
+  }
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int vec = H / 8;
+  for (int64_t p = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; p < total; p += nwarps) {
+    const int s = perm[p];
+    if (s < 0 || s >= R) {
+      if (lane == 0) atomicOr(status, MOE_DEVICE_ERR_CSR);
+      continue;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(s / k) * H);
+    uint4* dst = reinterpret_cast<uint4*>(Xp + p * H);
+    for (int c = lane; c < vec; c += 32) dst[c] = __ldg(src + c);
+  }
+}
+
+// out[t, :] = sum_j Y[t*k + j, :] in fp32, j ascending, rounded to bf16.
+__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ Y, int T, int H, int k,
+                                                      __nv_bfloat16* __restrict__ out) {
+  const int vec = H / 8;
+  const int64_t n = static_cast<int64_t>(T) * vec;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / vec;
+    const int c = static_cast<int>(i - t * vec);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(Y + (t * k + j) * H) + c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[2 * q] += bf16_lo(w[q]);
+        acc[2 * q + 1] += bf16_hi(w[q]);
+      }
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    reinterpret_cast<uint4*>(out + t * H)[c] = o;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_csr_count(const int32_t* idx, int R, int E, int32_t* chunk_counts, int* status,
+                             cudaStream_t stream) {
+  const int nchunks = csr_num_chunks(R);
+  if (nchunks == 0) return cudaSuccess;
+  csr_count_kernel<<<nchunks, kCsrThreads, E * sizeof(int), stream>>>(idx, R, E, chunk_counts, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_csr_scan(const int32_t* chunk_counts, int nchunks, int E, int32_t* chunk_base, int32_t* offsets,
+                            cudaStream_t stream) {
+  csr_scan_kernel<<<1, 1024, 0, stream>>>(chunk_counts, nchunks, E, chunk_base, offsets);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_csr_scatter(const int32_t* idx, int R, int E, const int32_t* chunk_base, int32_t* perm,
+                               int32_t* inv, cudaStream_t stream) {
+  const int nchunks = csr_num_chunks(R);
+  if (nchunks == 0) return cudaSuccess;
+  const size_t smem = static_cast<size_t>(kCsrWarps) * E * sizeof(int);
+  if (smem > 48 * 1024) {
+    cudaError_t err = cudaFuncSetAttribute(csr_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+  }
+  csr_scatter_kernel<<<nchunks, kCsrThreads, smem, stream>>>(idx, R, E, chunk_base, perm, inv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, const int32_t* offsets, int E, int R, int k,
+                          int H, __nv_bfloat16* Xp, int* status, int num_sms, cudaStream_t stream) {
+  if (R == 0) return cudaSuccess;
+  const int rows_per_block = 8;
+  const int blocks = static_cast<int>(std::min<int64_t>((R + rows_per_block - 1) / rows_per_block,
+                                                        static_cast<int64_t>(num_sms) * 16));
+  gather_rows_kernel<<<blocks, 256, 0, stream>>>(x, perm, offsets, E, R, k, H, Xp, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const __nv_bfloat16* Y, int T, int H, int k, __nv_bfloat16* out, int num_sms,
+                           cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const int64_t n = static_cast<int64_t>(T) * (H / 8);
+  const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(num_sms) * 16));
+  combine_kernel<<<blocks, 256, 0, stream>>>(Y, T, H, k, out);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

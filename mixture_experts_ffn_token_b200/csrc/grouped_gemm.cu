@@ -1,0 +1,545 @@
+// grouped_gemm.cu -- stages 3 and 4: the two grouped contractions over
+// stacked expert weights on the 5th-generation tensor cores.
+//
+//   gate_up:  h[p, :] = act(split(Xp[p, :] . W_gu[e] + b_gu[e]))   for p in
+//             expert e's segment [off[e], off[e+1]) of the permuted rows
+//             (StackedMoE gate_up_proj [E, H, 2D]; GatedActivation fused
+//             activations; concatenated or interleaved gate/up columns).
+//   down:     Y[perm[p], :] = w[perm[p]] * (h[p, :] . W_d[e] + b_d[e])
+//             (StackedMoE down_proj [E, D, H]; router weight after the expert,
+//             down bias weighted with it as in NeMo _apply_bias), stored at
+//             the slot row so the k-way combine reads tokens in order.
+//
+// Kernel design (one persistent CTA per SM, 192 threads):
+//   warp 0      TMA producer: for every tile and 64-wide K block, one 128x64
+//               box of A (K-major, 128-byte swizzle) and four 64x64 boxes of
+//               B (N-major, 128-byte swizzle) into a 4-stage ring, completion
+//               on a full[stage] mbarrier;
+//   warp 1      TMEM allocator and MMA issuer: one thread issues four
+//               tcgen05.mma 128x256x16 per stage (bf16 in, fp32 accumulate in
+//               TMEM) and tcgen05.commit's the stage back to the producer;
+//               two 256-column accumulators alternate between tiles;
+//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes (one output row
+//               per thread), bias + activation (gate_up) or bias x weight
+//               (down) in fp32, bf16 stores.
+// Tiles are the ragged expert segments cut in 128-row pieces times the
+// output columns; the per-expert piece counts are rebuilt from the CSR
+// offsets in shared memory at kernel start, and CTAs walk the tile list with
+// a static stride (expert-major, then output column block, then row piece,
+// so CTAs running together share a weight column block through L2).
+// Rows of a piece beyond its expert's segment are computed and discarded.
+// Weights are read in their stored [K, N] (N-contiguous) layout: the B
+// operand is MN-major, which tcgen05 supports for 16-bit types, so no
+// transposed copy of the weights is needed.  Every mbarrier wait is bounded
+// (mbar_wait); a timeout raises a CTA-wide abort, drains the copies and
+// MMAs in flight, frees TMEM and records MOE_DEVICE_ERR_TIMEOUT_* in the
+// status word.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;                 // rows per tile (TMEM lanes)
+constexpr int BN = 256;                 // accumulator columns per tile
+constexpr int BK = 64;                  // K per stage: one 128-byte swizzle row of bf16
+constexpr int UMMA_K = 16;              // K per tcgen05.mma (kind::f16)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;            // 16 KB
+constexpr int B_BOX_BYTES = BK * 64 * 2;        // 8 KB: 64 K rows x 64 N columns
+constexpr int B_BYTES = 4 * B_BOX_BYTES;        // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;             // two BN-column fp32 accumulators
+constexpr int CTRL_BYTES = 256;
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
+constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, /*a_mn_major=*/false, /*b_mn_major=*/true);
+
+constexpr int MODE_GATE_UP_CONCAT = 0;
+constexpr int MODE_GATE_UP_INTERLEAVED = 1;
+constexpr int MODE_DOWN = 2;
+
+struct GemmParams {
+  const int32_t* offsets;
+  const int32_t* perm;
+  const float* weights;
+  const __nv_bfloat16* bias;
+  __nv_bfloat16* out;
+  int* status;
+  int E, R, H, D;
+  int n_tiles, num_kb;
+  int activation;
+  float alpha, limit;
+  int err_bit;
+};
+
+struct TileCoord {
+  int e, row0, rows, n;
+};
+
+// Tile t -> (expert, first permuted row, valid rows, output column block).
+// s_mt is the exclusive prefix of per-expert 128-row pieces (s_mt[E] = total).
+__device__ __forceinline__ TileCoord decode_tile(int t, int n_tiles, int E, const int* s_mt, const int* s_off) {
+  int lo = 0, hi = E;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_mt[mid] * n_tiles <= t) lo = mid;
+    else hi = mid;
+  }
+  TileCoord c;
+  c.e = lo;
+  const int local = t - s_mt[lo] * n_tiles;
+  const int mt = s_mt[lo + 1] - s_mt[lo];
+  c.n = local / mt;
+  const int m = local - c.n * mt;
+  c.row0 = s_off[lo] + m * BM;
+  c.rows = min(BM, s_off[lo + 1] - c.row0);
+  return c;
+}
+
+__device__ __forceinline__ bool wait_time_only(uint32_t bar, uint32_t parity) {
+  int never = 0;
+  return mbar_wait(bar, parity, &never, kTimeoutNs);
+}
+
+// ----------------------------------------------------------- epilogues
+// gate_up, concatenated [gate | up]: accumulator columns 0..127 are gate
+// columns hcol0.., columns 128..255 the matching up columns.
+__device__ __forceinline__ void epilogue_gate_up_concat(const GemmParams& p, const TileCoord& tc, uint32_t tacc,
+                                                        int row) {
+  const bool valid = row < tc.rows;
+  const int hcol0 = tc.n * 128;
+  const int64_t prow = static_cast<int64_t>(tc.row0) + row;
+  const __nv_bfloat16* bg = p.bias != nullptr ? p.bias + static_cast<int64_t>(tc.e) * 2 * p.D : nullptr;
+#pragma unroll 1
+  for (int c = 0; c < 128; c += 16) {
+    uint32_t g[16], u[16];
+    tmem_ld16(tacc + c, g);
+    tmem_ld16(tacc + 128 + c, u);
+    tmem_ld_wait();
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int col = hcol0 + c + 8 * half;
+      if (valid && col < p.D) {
+        float hv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float gv = __uint_as_float(g[8 * half + j]);
+          float uv = __uint_as_float(u[8 * half + j]);
+          if (bg != nullptr) {
+            gv += __bfloat162float(bg[col + j]);
+            uv += __bfloat162float(bg[p.D + col + j]);
+          }
+          hv[j] = gated_act(p.activation, gv, uv, p.alpha, p.limit);
+        }
+        uint4 o;
+        o.x = pack_bf16x2(hv[0], hv[1]);
+        o.y = pack_bf16x2(hv[2], hv[3]);
+        o.z = pack_bf16x2(hv[4], hv[5]);
+        o.w = pack_bf16x2(hv[6], hv[7]);
+        *reinterpret_cast<uint4*>(p.out + prow * p.D + col) = o;
+      }
+    }
+  }
+}
+
+// gate_up, interleaved: accumulator columns (2j, 2j+1) are (gate, up) of h
+// column hcol0 + j.
+__device__ __forceinline__ void epilogue_gate_up_interleaved(const GemmParams& p, const TileCoord& tc, uint32_t tacc,
+                                                             int row) {
+  const bool valid = row < tc.rows;
+  const int hcol0 = tc.n * 128;
+  const int64_t prow = static_cast<int64_t>(tc.row0) + row;
+  const __nv_bfloat16* bg = p.bias != nullptr ? p.bias + static_cast<int64_t>(tc.e) * 2 * p.D : nullptr;
+#pragma unroll 1
+  for (int c = 0; c < 256; c += 32) {
+    uint32_t v[32];
+    tmem_ld16(tacc + c, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+    tmem_ld16(tacc + c + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+    tmem_ld_wait();
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int col = hcol0 + c / 2 + 8 * half;
+      if (valid && col < p.D) {
+        float hv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float gv = __uint_as_float(v[16 * half + 2 * j]);
+          float uv = __uint_as_float(v[16 * half + 2 * j + 1]);
+          if (bg != nullptr) {
+            gv += __bfloat162float(bg[2 * (col + j)]);
+            uv += __bfloat162float(bg[2 * (col + j) + 1]);
+          }
+          hv[j] = gated_act(p.activation, gv, uv, p.alpha, p.limit);
+        }
+        uint4 o;
+        o.x = pack_bf16x2(hv[0], hv[1]);
+        o.y = pack_bf16x2(hv[2], hv[3]);
+        o.z = pack_bf16x2(hv[4], hv[5]);
+        o.w = pack_bf16x2(hv[6], hv[7]);
+        *reinterpret_cast<uint4*>(p.out + prow * p.D + col) = o;
+      }
+    }
+  }
+}
+
+// down: (acc + b_d[e]) * w[slot], stored at the slot's row of Y.
+__device__ __forceinline__ void epilogue_down(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int row) {
+  bool ok = row < tc.rows;
+  int slot = 0;
+  float wgt = 0.f;
+  if (ok) {
+    slot = p.perm[tc.row0 + row];
+    if (slot < 0 || slot >= p.R) {
+      atomicOr(p.status, MOE_DEVICE_ERR_CSR);
+      ok = false;
+    } else {
+      wgt = p.weights[slot];
+    }
+  }
+  const int col0 = tc.n * BN;
+  const __nv_bfloat16* bd = p.bias != nullptr ? p.bias + static_cast<int64_t>(tc.e) * p.H : nullptr;
+  __nv_bfloat16* orow = p.out + static_cast<int64_t>(slot) * p.H;
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    uint32_t v[32];
+    tmem_ld16(tacc + c, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+    tmem_ld16(tacc + c + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+    tmem_ld_wait();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int col = col0 + c + 8 * q;
+      if (ok && col < p.H) {
+        float y[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float a = __uint_as_float(v[8 * q + j]);
+          if (bd != nullptr) a += __bfloat162float(bd[col + j]);
+          y[j] = a * wgt;
+        }
+        uint4 o;
+        o.x = pack_bf16x2(y[0], y[1]);
+        o.y = pack_bf16x2(y[2], y[3]);
+        o.z = pack_bf16x2(y[4], y[5]);
+        o.w = pack_bf16x2(y[6], y[7]);
+        *reinterpret_cast<uint4*>(orow + col) = o;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------- the kernel
+template <int MODE>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                        const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint8_t* ctrl = smem + STAGES * STAGE_BYTES;
+  const uint32_t full0 = smem_u32(ctrl);              // STAGES mbarriers
+  const uint32_t empty0 = full0 + 8 * STAGES;         // STAGES mbarriers
+  const uint32_t tfull0 = empty0 + 8 * STAGES;        // 2 mbarriers
+  const uint32_t tempty0 = tfull0 + 16;               // 2 mbarriers
+  const uint32_t drain_bar = tempty0 + 16;            // 1 mbarrier
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 128);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 132);
+  int* bad_flag = reinterpret_cast<int*>(ctrl + 136);
+  int* s_off = reinterpret_cast<int*>(ctrl + CTRL_BYTES);
+  int* s_mt = s_off + (p.E + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 128);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *bad_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_map(&mapA);
+    tma_prefetch_map(&mapB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) s_off[i] = p.offsets[i];
+  __syncthreads();
+  if (warp == 0) {
+    // Validate the CSR and build the per-expert prefix of 128-row pieces.
+    const int per = (p.E + 31) / 32;
+    const int e0 = min(lane * per, p.E), e1 = min(e0 + per, p.E);
+    int local = 0;
+    bool bad = false;
+    for (int e = e0; e < e1; ++e) {
+      const int cnt = s_off[e + 1] - s_off[e];
+      if (cnt < 0) bad = true;
+      else local += (cnt + BM - 1) / BM;
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    int run = incl - local;
+    for (int e = e0; e < e1; ++e) {
+      s_mt[e] = run;
+      const int cnt = s_off[e + 1] - s_off[e];
+      if (cnt > 0) run += (cnt + BM - 1) / BM;
+    }
+    if (lane == 31) s_mt[p.E] = incl;
+    if (lane == 0 && (s_off[0] != 0 || s_off[p.E] > p.R)) bad = true;
+    if (__any_sync(0xffffffffu, bad) && lane == 0) *bad_flag = 1;
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  const bool bad = *bad_flag != 0;
+  if (bad && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, MOE_DEVICE_ERR_CSR);
+  const int total_tiles = bad ? 0 : s_mt[p.E] * p.n_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+        const TileCoord tc = decode_tile(t, p.n_tiles, p.E, s_mt, s_off);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t ph = static_cast<uint32_t>(it / STAGES) & 1u;
+          if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sbase + s * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+          const uint32_t fb = full0 + 8 * s;
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          tma_load_2d(sa, &mapA, fb, kb * BK, tc.row0);
+          if constexpr (MODE == MODE_GATE_UP_CONCAT) {
+            // 4-D view {D, 2 (gate/up), H, E}: two gate boxes then two up boxes.
+            const int c0 = tc.n * 128;
+            tma_load_4d(sb, &mapB, fb, c0, 0, kb * BK, tc.e);
+            tma_load_4d(sb + B_BOX_BYTES, &mapB, fb, c0 + 64, 0, kb * BK, tc.e);
+            tma_load_4d(sb + 2 * B_BOX_BYTES, &mapB, fb, c0, 1, kb * BK, tc.e);
+            tma_load_4d(sb + 3 * B_BOX_BYTES, &mapB, fb, c0 + 64, 1, kb * BK, tc.e);
+          } else {
+            // 3-D view {N, K, E}: four consecutive 64-column boxes.
+            const int c0 = tc.n * BN;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * B_BOX_BYTES, &mapB, fb, c0 + 64 * j, kb * BK, tc.e);
+          }
+          ++it;
+        }
+      }
+      if (ok) {
+        // Tail: wait until the MMA warp has released every stage, so that no
+        // tcgen05.commit arrival lands after this CTA exits.
+        for (int i = 0; i < STAGES; ++i, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = static_cast<uint32_t>(it / STAGES) & 1u;
+          if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kTimeoutNs)) break;
+        }
+      } else {
+        // Aborted: let the copies already issued land before shared memory
+        // is released (time-bounded, independent of the abort flag).
+        for (int s = 0; s < STAGES; ++s) {
+          if (it > s) {
+            const int last = s + ((it - 1 - s) / STAGES) * STAGES;
+            wait_time_only(full0 + 8 * s, static_cast<uint32_t>(last / STAGES) & 1u);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // --------------------------------------------------- MMA issuer
+      int it = 0, ti = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x, ++ti) {
+        const int acc = ti & 1;
+        const uint32_t aph = static_cast<uint32_t>(ti >> 1) & 1u;
+        if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, abort_flag, kTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t ph = static_cast<uint32_t>(it / STAGES) & 1u;
+          if (!mbar_wait(full0 + 8 * s, ph, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t sa = sbase + s * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            // A: K-major rows of 128 B, 8-row swizzle atoms 1024 B apart; a
+            // 16-wide K step is 32 B along the row.
+            const uint64_t a_desc = smem_desc_sw128(sa + kk * UMMA_K * 2, 16, 1024);
+            // B: N-major; 64-column blocks B_BOX_BYTES apart (LBO), 8-row K
+            // groups 1024 B apart (SBO); a 16-row K step is 2048 B.
+            const uint64_t b_desc = smem_desc_sw128(sb + kk * UMMA_K * 128, B_BOX_BYTES, 1024);
+            mma_bf16_ss(d_tmem, a_desc, b_desc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(empty0 + 8 * s);
+          ++it;
+        }
+        if (!ok) break;
+        mma_commit(tfull0 + 8 * acc);
+      }
+      if (!ok) {
+        // Aborted: every MMA issued so far must finish before TMEM is freed.
+        mma_commit(drain_bar);
+        wait_time_only(drain_bar, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------ epilogue
+    const int quad = warp & 3;  // this warp may access TMEM lanes 32*quad..+31
+    const int row = quad * 32 + lane;
+    int ti = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++ti) {
+      const TileCoord tc = decode_tile(t, p.n_tiles, p.E, s_mt, s_off);
+      const int acc = ti & 1;
+      const uint32_t aph = static_cast<uint32_t>(ti >> 1) & 1u;
+      const bool got = mbar_wait(tfull0 + 8 * acc, aph, abort_flag, kTimeoutNs);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after_sync();
+      const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
+      if constexpr (MODE == MODE_GATE_UP_CONCAT) epilogue_gate_up_concat(p, tc, tacc, row);
+      else if constexpr (MODE == MODE_GATE_UP_INTERLEAVED) epilogue_gate_up_interleaved(p, tc, tacc, row);
+      else epilogue_down(p, tc, tacc, row);
+      tc_fence_before_sync();
+      mbar_arrive(tempty0 + 8 * acc);
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, p.err_bit);
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+bool encode_bf16_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                     const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  auto enc = encoder();
+  if (enc == nullptr) return false;
+  const cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
+                         dims, strides_bytes, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+constexpr size_t smem_bytes_for(int E) {
+  return 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + CTRL_BYTES + 2 * static_cast<size_t>(E + 1) * 4;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t stream) {
+  if (a.R == 0) return cudaSuccess;
+  const bool down = MODE == MODE_DOWN;
+  const int K = down ? a.D : a.H;
+  CUtensorMap mapA, mapB;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(a.R)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {64, BM};
+    if (!encode_bf16_map(&mapA, a.A, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  const cuuint64_t H = a.H, D = a.D, E = a.E;
+  if (MODE == MODE_GATE_UP_CONCAT) {
+    const cuuint64_t dims[4] = {D, 2, H, E};
+    const cuuint64_t strides[3] = {D * 2, 2 * D * 2, H * 2 * D * 2};
+    const cuuint32_t box[4] = {64, 1, BK, 1};
+    if (!encode_bf16_map(&mapB, a.W, 4, dims, strides, box)) return cudaErrorInvalidValue;
+  } else if (MODE == MODE_GATE_UP_INTERLEAVED) {
+    const cuuint64_t dims[3] = {2 * D, H, E};
+    const cuuint64_t strides[2] = {2 * D * 2, H * 2 * D * 2};
+    const cuuint32_t box[3] = {64, BK, 1};
+    if (!encode_bf16_map(&mapB, a.W, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  } else {
+    const cuuint64_t dims[3] = {H, D, E};
+    const cuuint64_t strides[2] = {H * 2, D * H * 2};
+    const cuuint32_t box[3] = {64, BK, 1};
+    if (!encode_bf16_map(&mapB, a.W, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  GemmParams p;
+  p.offsets = a.offsets;
+  p.perm = a.perm;
+  p.weights = a.weights;
+  p.bias = a.bias;
+  p.out = a.out;
+  p.status = a.status;
+  p.E = a.E;
+  p.R = a.R;
+  p.H = a.H;
+  p.D = a.D;
+  p.n_tiles = down ? (a.H + BN - 1) / BN : (a.D + 127) / 128;
+  p.num_kb = (K + BK - 1) / BK;
+  p.activation = a.activation;
+  p.alpha = a.alpha;
+  p.limit = a.limit;
+  p.err_bit = down ? MOE_DEVICE_ERR_TIMEOUT_GEMM2 : MOE_DEVICE_ERR_TIMEOUT_GEMM1;
+  const int64_t max_pieces = a.R / BM + std::min(a.E, a.R);
+  const int64_t max_tiles = max_pieces * p.n_tiles;
+  const int grid = static_cast<int>(std::min<int64_t>(max_tiles, a.num_sms));
+  const size_t smem = smem_bytes_for(a.E);
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_bytes_for(kMaxExperts)));
+  if (err != cudaSuccess) return err;
+  grouped_gemm_kernel<MODE><<<grid, NUM_THREADS, smem, stream>>>(mapA, mapB, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tensor_map_encoder_available() { return encoder() != nullptr; }
+
+cudaError_t launch_gemm_gate_up(const GroupedGemmArgs& a, cudaStream_t stream) {
+  return a.gate_up_format == 0 ? launch_mode<MODE_GATE_UP_CONCAT>(a, stream)
+                               : launch_mode<MODE_GATE_UP_INTERLEAVED>(a, stream);
+}
+
+cudaError_t launch_gemm_down(const GroupedGemmArgs& a, cudaStream_t stream) {
+  return launch_mode<MODE_DOWN>(a, stream);
+}
+
+}  // namespace moe

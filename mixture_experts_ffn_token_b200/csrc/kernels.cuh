@@ -1,0 +1,70 @@
+// kernels.cuh -- launchers of the sm_100a kernels, called by the C ABI
+// (moe_api.cu).  Every launcher only enqueues work on `stream` and returns
+// the launch status.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// ------------------------------------------------------------------ router
+struct RouterArgs {
+  const void* logits;
+  int logits_bf16;
+  int64_t stride;
+  int T, E, k, S;
+  int sink;                  // 0 softmax top-k, 1 sigmoid + sink lanes
+  const float* expert_bias;  // [E] or null
+  const float* global_scale; // device [1] or null
+  float route_scale;
+  int32_t* idx;              // [T,k]
+  float* w;                  // [T,k]
+  float* sink_w;             // [T,S] or null
+  int* status_reset;         // zeroed by the first thread, or null
+};
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------------- CSR
+constexpr int kCsrChunk = 2048;      // slots per CTA
+constexpr int kCsrThreads = 512;     // 16 warps x 128 slots
+inline int csr_num_chunks(int64_t R) { return static_cast<int>((R + kCsrChunk - 1) / kCsrChunk); }
+cudaError_t launch_csr_count(const int32_t* idx, int R, int E, int32_t* chunk_counts, int* status,
+                             cudaStream_t stream);
+cudaError_t launch_csr_scan(const int32_t* chunk_counts, int nchunks, int E, int32_t* chunk_base,
+                            int32_t* offsets, cudaStream_t stream);
+cudaError_t launch_csr_scatter(const int32_t* idx, int R, int E, const int32_t* chunk_base, int32_t* perm,
+                               int32_t* inv, cudaStream_t stream);
+
+// ----------------------------------------------------- gather and combine
+cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, const int32_t* offsets, int E, int R,
+                          int k, int H, __nv_bfloat16* Xp, int* status, int num_sms, cudaStream_t stream);
+cudaError_t launch_combine(const __nv_bfloat16* Y, int T, int H, int k, __nv_bfloat16* out, int num_sms,
+                           cudaStream_t stream);
+
+// ------------------------------------------------------------ grouped GEMM
+struct GroupedGemmArgs {
+  // routing (device)
+  const int32_t* offsets;   // [E+1]
+  const int32_t* perm;      // [R]
+  const float* weights;     // [R] routing weight per slot (down GEMM)
+  int E, R, T, k;
+  // problem
+  int H, D;
+  int gate_up_format;       // 0 concatenated, 1 interleaved
+  int activation;           // 0 silu, 1 swigluoai, 2 gelu_tanh
+  float alpha, limit;
+  // operands (device)
+  const __nv_bfloat16* A;   // Xp [R,H] (gate_up) or h [R,D] (down)
+  const __nv_bfloat16* W;   // [E,H,2D] (gate_up) or [E,D,H] (down)
+  const __nv_bfloat16* bias;// [E,2D] / [E,H] or null
+  __nv_bfloat16* out;       // h [R,D] (gate_up) or Y [R,H] slot rows (down)
+  int* status;
+  int num_sms;
+};
+cudaError_t launch_gemm_gate_up(const GroupedGemmArgs& a, cudaStream_t stream);
+cudaError_t launch_gemm_down(const GroupedGemmArgs& a, cudaStream_t stream);
+
+// Resolves cuTensorMapEncodeTiled through the runtime (no libcuda link).
+bool tensor_map_encoder_available();
+
+}  // namespace moe

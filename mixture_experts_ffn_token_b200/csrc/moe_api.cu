@@ -1,0 +1,381 @@
+// moe_api.cu -- the C ABI declared in include/moe.h: host-side validation,
+// the workspace layout and the launch sequence of each entry point.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.cuh"
+
+using moe::kMaxExperts;
+using moe::kMaxTopK;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool checked = false;
+  bool supported = false;
+  int num_sms = 0;
+};
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_devices_mu;
+
+// The current device must be compute capability 10.0 (the library's code is
+// sm_100a only) and the driver must expose the tensor-map encoder.
+moe_status_t current_device(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_devices_mu);
+  DeviceInfo& d = g_devices[dev];
+  if (!d.checked) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    d.supported = major == 10 && minor == 0 && moe::tensor_map_encoder_available();
+    d.num_sms = sms;
+    d.checked = true;
+  }
+  if (!d.supported) return MOE_ERR_UNSUPPORTED;
+  *num_sms = d.num_sms;
+  return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status_t validate_config(const moe_config_t* c) {
+  if (c == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  if (c->num_tokens < 0 || c->hidden_dim <= 0 || c->num_experts <= 0 || c->top_k <= 0 || c->moe_dim <= 0 ||
+      c->num_sink < 0)
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (c->top_k > c->num_experts) return MOE_ERR_INVALID_ARGUMENT;
+  if (c->router != MOE_ROUTER_SOFTMAX_TOPK && c->router != MOE_ROUTER_SIGMOID_SINK) return MOE_ERR_INVALID_ARGUMENT;
+  if (c->logits_dtype != MOE_DTYPE_BF16 && c->logits_dtype != MOE_DTYPE_F32) return MOE_ERR_INVALID_ARGUMENT;
+  if (c->gate_up_format != MOE_GATE_UP_CONCATENATED && c->gate_up_format != MOE_GATE_UP_INTERLEAVED)
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (c->activation != MOE_ACT_SILU && c->activation != MOE_ACT_SWIGLUOAI && c->activation != MOE_ACT_GELU_TANH)
+    return MOE_ERR_INVALID_ARGUMENT;
+  // GatedActivation: alpha must be 0 unless swigluoai; limit must be 0 for
+  // gelu_tanh; a negative clamp bound is meaningless.
+  if (!std::isfinite(c->alpha) || !std::isfinite(c->limit) || c->limit < 0.f) return MOE_ERR_INVALID_ARGUMENT;
+  if (c->alpha != 0.f && c->activation != MOE_ACT_SWIGLUOAI) return MOE_ERR_INVALID_ARGUMENT;
+  if (c->limit != 0.f && c->activation == MOE_ACT_GELU_TANH) return MOE_ERR_INVALID_ARGUMENT;
+  if (c->has_bias != 0 && c->has_bias != 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (c->router == MOE_ROUTER_SOFTMAX_TOPK && c->num_sink != 0) return MOE_ERR_INVALID_ARGUMENT;
+  if (c->logits_row_stride < static_cast<int64_t>(c->num_experts) + c->num_sink) return MOE_ERR_INVALID_ARGUMENT;
+  if (c->router == MOE_ROUTER_SIGMOID_SINK && !std::isfinite(c->route_scale)) return MOE_ERR_INVALID_ARGUMENT;
+  // What this library implements.
+  if (c->num_experts > kMaxExperts || c->top_k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+  if (c->hidden_dim % 8 != 0 || c->moe_dim % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (c->router == MOE_ROUTER_SIGMOID_SINK) {
+    // sink_gate_router_kernel: top-k plus sink lanes must be a power of two
+    // no greater than the warp size.
+    const int n = c->top_k + c->num_sink;
+    if (n > 32 || (n & (n - 1)) != 0) return MOE_ERR_UNSUPPORTED;
+  }
+  const int64_t R = static_cast<int64_t>(c->num_tokens) * c->top_k;
+  if (R > (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+  const int64_t pieces = R / 128 + c->num_experts;
+  const int64_t ntiles = std::max<int64_t>((c->moe_dim + 127) / 128, (c->hidden_dim + 255) / 256);
+  if (pieces * ntiles > (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t status, chunk_counts, chunk_base, offsets, perm, idx, w, sink, xp, h, total;
+};
+
+WsLayout ws_layout(const moe_config_t* c) {
+  const size_t T = static_cast<size_t>(c->num_tokens), H = c->hidden_dim, E = c->num_experts, D = c->moe_dim;
+  const size_t R = T * c->top_k;
+  const size_t nchunks = static_cast<size_t>(moe::csr_num_chunks(static_cast<int64_t>(R)));
+  WsLayout L;
+  size_t o = 0;
+  L.status = o;
+  o += 256;
+  L.chunk_counts = o;
+  o += align256(nchunks * E * 4);
+  L.chunk_base = o;
+  o += align256(nchunks * E * 4);
+  L.offsets = o;
+  o += align256((E + 1) * 4);
+  L.perm = o;
+  o += align256(R * 4);
+  L.idx = o;
+  o += align256(R * 4);
+  L.w = o;
+  o += align256(R * 4);
+  L.sink = o;
+  o += align256(T * static_cast<size_t>(c->num_sink) * 4);
+  L.xp = o;  // Xp [R, H] for the gate_up GEMM, then Y [R, H] from the down GEMM
+  o += align256(R * H * 2);
+  L.h = o;
+  o += align256(R * D * 2);
+  L.total = o;
+  return L;
+}
+
+template <typename T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(base) + off);
+}
+
+moe_status_t check_workspace(const moe_config_t* c, const void* ws, size_t bytes, WsLayout* L) {
+  *L = ws_layout(c);
+  if (ws == nullptr || !aligned16(ws)) return MOE_ERR_INVALID_ARGUMENT;
+  if (bytes < L->total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  return MOE_OK;
+}
+
+moe_status_t check_bias(const moe_config_t* c, const void* gate_up_b, const void* down_b) {
+  if (c->has_bias) return (gate_up_b != nullptr && down_b != nullptr) ? MOE_OK : MOE_ERR_INVALID_ARGUMENT;
+  return (gate_up_b == nullptr && down_b == nullptr) ? MOE_OK : MOE_ERR_INVALID_ARGUMENT;
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+moe::RouterArgs router_args(const moe_config_t* c, const void* logits, const float* bias, const float* gscale,
+                            int32_t* idx, float* w, float* sink_w, int* status_reset) {
+  moe::RouterArgs a;
+  a.logits = logits;
+  a.logits_bf16 = c->logits_dtype == MOE_DTYPE_BF16;
+  a.stride = c->logits_row_stride;
+  a.T = c->num_tokens;
+  a.E = c->num_experts;
+  a.k = c->top_k;
+  a.S = c->num_sink;
+  a.sink = c->router == MOE_ROUTER_SIGMOID_SINK;
+  a.expert_bias = a.sink ? bias : nullptr;
+  a.global_scale = a.sink ? gscale : nullptr;
+  a.route_scale = c->route_scale;
+  a.idx = idx;
+  a.w = w;
+  a.sink_w = sink_w;
+  a.status_reset = status_reset;
+  return a;
+}
+
+// Gather -> gate_up GEMM -> down GEMM -> combine.  ev (may be null) gets a
+// record before each of the four kernels and after the last.
+moe_status_t enqueue_ffn(const moe_config_t* c, const void* x, const void* gate_up_w, const void* gate_up_b,
+                         const void* down_w, const void* down_b, const int32_t* offsets, const int32_t* perm,
+                         const float* weights, void* out, void* ws, const WsLayout& L, int num_sms,
+                         cudaStream_t stream, cudaEvent_t const* ev) {
+  const int T = c->num_tokens, H = c->hidden_dim, E = c->num_experts, k = c->top_k, D = c->moe_dim;
+  const int R = T * k;
+  int* status = at<int>(ws, L.status);
+  __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
+  __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
+  auto rec = [&](int i) {
+    if (ev != nullptr) cudaEventRecord(ev[i], stream);
+  };
+  rec(0);
+  cudaError_t err = moe::launch_gather(static_cast<const __nv_bfloat16*>(x), perm, offsets, E, R, k, H, xp, status,
+                                       num_sms, stream);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  moe::GroupedGemmArgs g;
+  g.offsets = offsets;
+  g.perm = perm;
+  g.weights = weights;
+  g.E = E;
+  g.R = R;
+  g.T = T;
+  g.k = k;
+  g.H = H;
+  g.D = D;
+  g.gate_up_format = c->gate_up_format;
+  g.activation = c->activation;
+  g.alpha = c->alpha;
+  g.limit = c->limit;
+  g.status = status;
+  g.num_sms = num_sms;
+  g.A = xp;
+  g.W = static_cast<const __nv_bfloat16*>(gate_up_w);
+  g.bias = static_cast<const __nv_bfloat16*>(gate_up_b);
+  g.out = h;
+  rec(1);
+  err = moe::launch_gemm_gate_up(g, stream);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  g.A = h;
+  g.W = static_cast<const __nv_bfloat16*>(down_w);
+  g.bias = static_cast<const __nv_bfloat16*>(down_b);
+  g.out = xp;  // Y reuses the Xp region: the gate_up GEMM has finished with it
+  rec(2);
+  err = moe::launch_gemm_down(g, stream);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  rec(3);
+  err = moe::launch_combine(xp, T, H, k, static_cast<__nv_bfloat16*>(out), num_sms, stream);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  rec(4);
+  return MOE_OK;
+}
+
+moe_status_t enqueue_csr(const moe_config_t* c, const int32_t* idx, int32_t* offsets, int32_t* perm, int32_t* inv,
+                         void* ws, const WsLayout& L, cudaStream_t stream, cudaEvent_t const* ev) {
+  const int R = c->num_tokens * c->top_k, E = c->num_experts;
+  auto rec = [&](int i) {
+    if (ev != nullptr) cudaEventRecord(ev[i], stream);
+  };
+  rec(0);
+  if (moe::launch_csr_count(idx, R, E, at<int32_t>(ws, L.chunk_counts), at<int>(ws, L.status), stream) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  rec(1);
+  if (moe::launch_csr_scan(at<int32_t>(ws, L.chunk_counts), moe::csr_num_chunks(R), E, at<int32_t>(ws, L.chunk_base),
+                           offsets, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  rec(2);
+  if (moe::launch_csr_scatter(idx, R, E, at<int32_t>(ws, L.chunk_base), perm, inv, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const void* logits, const float* expert_bias,
+                          const float* global_scale, const void* gate_up_w, const void* gate_up_b,
+                          const void* down_w, const void* down_b, void* out, int32_t* idx_out, float* w_out,
+                          float* sink_out, void* ws, size_t ws_bytes, cudaStream_t stream, cudaEvent_t const* ev) {
+  moe_status_t st = validate_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->num_tokens == 0) return MOE_OK;  // nothing to read or write; empty tensors may have null pointers
+  if (x == nullptr || logits == nullptr || gate_up_w == nullptr || down_w == nullptr || out == nullptr)
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(gate_up_w) || !aligned16(down_w) || !aligned16(out))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if ((st = check_bias(cfg, gate_up_b, down_b)) != MOE_OK) return st;
+  WsLayout L;
+  if ((st = check_workspace(cfg, ws, ws_bytes, &L)) != MOE_OK) return st;
+  int num_sms = 0;
+  if ((st = current_device(&num_sms)) != MOE_OK) return st;
+
+  int32_t* idx = idx_out != nullptr ? idx_out : at<int32_t>(ws, L.idx);
+  float* w = w_out != nullptr ? w_out : at<float>(ws, L.w);
+  float* sink = (sink_out != nullptr || cfg->num_sink == 0) ? sink_out : at<float>(ws, L.sink);
+  if (ev != nullptr) cudaEventRecord(ev[0], stream);
+  const moe::RouterArgs ra = router_args(cfg, logits, expert_bias, global_scale, idx, w, sink, at<int>(ws, L.status));
+  if (moe::launch_router(ra, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  if ((st = enqueue_csr(cfg, idx, offsets, perm, nullptr, ws, L, stream, ev != nullptr ? ev + 1 : nullptr)) != MOE_OK)
+    return st;
+  return enqueue_ffn(cfg, x, gate_up_w, gate_up_b, down_w, down_b, offsets, perm, w, out, ws, L, num_sms, stream,
+                     ev != nullptr ? ev + 4 : nullptr);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARGUMENT: return "MOE_ERR_INVALID_ARGUMENT";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "MOE_ERR_WORKSPACE_TOO_SMALL";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
+  const moe_status_t st = validate_config(cfg);
+  if (st != MOE_OK) return st;
+  if (bytes == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  *bytes = ws_layout(cfg).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_route(const moe_config_t* cfg, const void* logits, const float* expert_bias,
+                       const float* global_scale, int32_t* expert_indices, float* expert_weights,
+                       float* sink_weights, moe_stream_t stream) {
+  moe_status_t st = validate_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->num_tokens == 0) return MOE_OK;
+  if (logits == nullptr || expert_indices == nullptr || expert_weights == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  if (cfg->router == MOE_ROUTER_SIGMOID_SINK && cfg->num_sink > 0 && sink_weights == nullptr)
+    return MOE_ERR_INVALID_ARGUMENT;
+  int num_sms = 0;
+  if ((st = current_device(&num_sms)) != MOE_OK) return st;
+  const moe::RouterArgs ra =
+      router_args(cfg, logits, expert_bias, global_scale, expert_indices, expert_weights, sink_weights, nullptr);
+  return cuda_status(moe::launch_router(ra, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_create_indices(const moe_config_t* cfg, const int32_t* expert_indices, int32_t* expert_offsets,
+                                int32_t* permutation, int32_t* inverse, void* workspace, size_t workspace_bytes,
+                                moe_stream_t stream) {
+  moe_status_t st = validate_config(cfg);
+  if (st != MOE_OK) return st;
+  if (expert_offsets == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  if (cfg->num_tokens > 0 && (expert_indices == nullptr || permutation == nullptr)) return MOE_ERR_INVALID_ARGUMENT;
+  WsLayout L;
+  if ((st = check_workspace(cfg, workspace, workspace_bytes, &L)) != MOE_OK) return st;
+  int num_sms = 0;
+  if ((st = current_device(&num_sms)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+  return enqueue_csr(cfg, expert_indices, expert_offsets, permutation, inverse, workspace, L, s, nullptr);
+}
+
+moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x, const void* gate_up_w, const void* gate_up_b,
+                             const void* down_w, const void* down_b, const int32_t* expert_offsets,
+                             const int32_t* permutation, const float* expert_weights, void* out, void* workspace,
+                             size_t workspace_bytes, moe_stream_t stream) {
+  moe_status_t st = validate_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->num_tokens == 0) return MOE_OK;
+  if (x == nullptr || gate_up_w == nullptr || down_w == nullptr || out == nullptr || expert_offsets == nullptr ||
+      permutation == nullptr || expert_weights == nullptr)
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(gate_up_w) || !aligned16(down_w) || !aligned16(out))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if ((st = check_bias(cfg, gate_up_b, down_b)) != MOE_OK) return st;
+  WsLayout L;
+  if ((st = check_workspace(cfg, workspace, workspace_bytes, &L)) != MOE_OK) return st;
+  int num_sms = 0;
+  if ((st = current_device(&num_sms)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+  return enqueue_ffn(cfg, x, gate_up_w, gate_up_b, down_w, down_b, expert_offsets, permutation, expert_weights, out,
+                     workspace, L, num_sms, s, nullptr);
+}
+
+moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* logits, const float* expert_bias,
+                         const float* global_scale, const void* gate_up_w, const void* gate_up_b, const void* down_w,
+                         const void* down_b, void* out, int32_t* expert_indices_out, float* expert_weights_out,
+                         float* sink_weights_out, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  return forward_impl(cfg, x, logits, expert_bias, global_scale, gate_up_w, gate_up_b, down_w, down_b, out,
+                      expert_indices_out, expert_weights_out, sink_weights_out, workspace, workspace_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+moe_status_t moe_forward_timed(const moe_config_t* cfg, const void* x, const void* logits, const float* expert_bias,
+                               const float* global_scale, const void* gate_up_w, const void* gate_up_b,
+                               const void* down_w, const void* down_b, void* out, int32_t* expert_indices_out,
+                               float* expert_weights_out, float* sink_weights_out, void* workspace,
+                               size_t workspace_bytes, moe_stream_t stream, void* const* stage_events) {
+  if (stage_events == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  for (int i = 0; i < MOE_NUM_STAGE_EVENTS; ++i)
+    if (stage_events[i] == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  return forward_impl(cfg, x, logits, expert_bias, global_scale, gate_up_w, gate_up_b, down_w, down_b, out,
+                      expert_indices_out, expert_weights_out, sink_weights_out, workspace, workspace_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<cudaEvent_t const*>(stage_events));
+}
+
+moe_status_t moe_device_status(const void* workspace, int32_t* device_status, moe_stream_t stream) {
+  if (workspace == nullptr || device_status == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  *device_status = v;
+  if (v & (MOE_DEVICE_ERR_TIMEOUT_GEMM1 | MOE_DEVICE_ERR_TIMEOUT_GEMM2)) return MOE_ERR_DEVICE_TIMEOUT;
+  return MOE_OK;
+}
+
+}  // extern "C"

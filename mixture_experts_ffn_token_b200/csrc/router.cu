@@ -1,0 +1,155 @@
+// router.cu -- stage 1: one warp per token.
+//
+// Softmax top-k router: the k largest logits, ties to the lowest expert
+// index, ordered by descending logit; weights = softmax over the k selected
+// logits (the StackedMoE page names the gate but not its body; this is the
+// plain top-k softmax reading).
+//
+// Sigmoid-gate router with sink lanes (Mojo sink_gate_router_kernel page,
+// description and Args): selection score sigmoid(z) + expert_bias (bias for
+// selection only), top-k on that score, then a softmax over the log-sigmoid
+// of the selected experts' RAW logits concatenated with the S always-on sink
+// logits, times route_scale * global_scale.  The page computes this in log
+// space so it stays finite where the sigmoids underflow; so does this kernel.
+//
+// Design: the page's kernel uses one block per token and one thread per
+// expert with a block-level top-k.  Here one warp owns a token: each lane
+// holds ceil(E/32) scores in registers, the k winners are found by k rounds
+// of a 5-step shuffle arg-max (ties -> lower index), and lanes 0..k+S-1 then
+// hold one normalisation entry each, so the final softmax is one warp
+// reduction.  The selection score is the fp32 value fl32(sigmoid(z)) + b
+// (sigmoid evaluated in fp64 and rounded once), so the choice is decided in
+// single precision exactly as the oracle decides it; the weights are
+// evaluated in fp64 and rounded to fp32 on store.
+#include <climits>
+
+#include "kernels.cuh"
+
+namespace moe {
+namespace {
+
+template <bool BF16>
+__device__ __forceinline__ float load_logit(const void* logits, int64_t i) {
+  if constexpr (BF16) {
+    return __bfloat162float(static_cast<const __nv_bfloat16*>(logits)[i]);
+  } else {
+    return static_cast<const float*>(logits)[i];
+  }
+}
+
+__device__ __forceinline__ double log_sigmoid(double z) { return fmin(z, 0.0) - log1p(exp(-fabs(z))); }
+
+template <int NPL, bool SINK, bool BF16>
+__global__ void __launch_bounds__(128) router_kernel(const RouterArgs a) {
+  if (a.status_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.status_reset = 0;
+  const int lane = threadIdx.x & 31;
+  const int t = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
+  if (t >= a.T) return;
+  const int64_t row = static_cast<int64_t>(t) * a.stride;
+
+  float key[NPL];
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int e = lane + 32 * i;
+    float kv = -INFINITY;
+    if (e < a.E) {
+      const float z = load_logit<BF16>(a.logits, row + e);
+      if constexpr (SINK) {
+        const float sig = static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(z))));
+        const float b = a.expert_bias != nullptr ? a.expert_bias[e] : 0.f;
+        kv = __fadd_rn(sig, b);
+      } else {
+        kv = z;
+      }
+    }
+    key[i] = kv;
+  }
+
+  uint32_t taken = 0;
+  int my_e = 0;
+  for (int j = 0; j < a.k; ++j) {
+    float bv = -INFINITY;
+    int bi = INT_MAX;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < a.E && !((taken >> i) & 1u)) {
+        if (key[i] > bv || (key[i] == bv && e < bi)) {
+          bv = key[i];
+          bi = e;
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    // bi == INT_MAX only for NaN scores: the index is then left out of range
+    // and the CSR build flags it.
+    if (bi < a.E && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == j) my_e = bi;
+  }
+
+  const int n_norm = a.k + (SINK ? a.S : 0);
+  const bool active = lane < n_norm;
+  double v = -INFINITY;
+  if (lane < a.k) {
+    const float z = my_e < a.E ? load_logit<BF16>(a.logits, row + my_e) : NAN;
+    v = SINK ? log_sigmoid(static_cast<double>(z)) : static_cast<double>(z);
+  } else if (SINK && active) {
+    v = log_sigmoid(static_cast<double>(load_logit<BF16>(a.logits, row + a.E + (lane - a.k))));
+  }
+  double m = v;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+  const double ex = active ? exp(v - m) : 0.0;
+  double sum = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  double w = ex / sum;
+  if (SINK) {
+    const double gs = a.global_scale != nullptr ? static_cast<double>(*a.global_scale) : 1.0;
+    w *= static_cast<double>(a.route_scale) * gs;
+  }
+  if (lane < a.k) {
+    a.idx[static_cast<int64_t>(t) * a.k + lane] = my_e;
+    a.w[static_cast<int64_t>(t) * a.k + lane] = static_cast<float>(w);
+  } else if (SINK && active) {
+    a.sink_w[static_cast<int64_t>(t) * a.S + (lane - a.k)] = static_cast<float>(w);
+  }
+}
+
+template <int NPL>
+cudaError_t launch_npl(const RouterArgs& a, cudaStream_t stream) {
+  const int warps_per_block = 4;
+  const dim3 grid((a.T + warps_per_block - 1) / warps_per_block);
+  const dim3 block(32 * warps_per_block);
+  if (a.sink) {
+    if (a.logits_bf16) router_kernel<NPL, true, true><<<grid, block, 0, stream>>>(a);
+    else router_kernel<NPL, true, false><<<grid, block, 0, stream>>>(a);
+  } else {
+    if (a.logits_bf16) router_kernel<NPL, false, true><<<grid, block, 0, stream>>>(a);
+    else router_kernel<NPL, false, false><<<grid, block, 0, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t stream) {
+  if (a.T <= 0) return cudaSuccess;
+  const int per_lane = (a.E + 31) / 32;
+  if (per_lane <= 1) return launch_npl<1>(a, stream);
+  if (per_lane <= 2) return launch_npl<2>(a, stream);
+  if (per_lane <= 4) return launch_npl<4>(a, stream);
+  if (per_lane <= 8) return launch_npl<8>(a, stream);
+  if (per_lane <= 16) return launch_npl<16>(a, stream);
+  return launch_npl<32>(a, stream);
+}
+
+}  // namespace moe

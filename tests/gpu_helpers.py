@@ -1,0 +1,90 @@
+"""Shared pieces of the GPU parity tests: run the CUDA path through the C ABI
+and compute the matching fp64 oracle result on the same seeded inputs."""
+import numpy as np
+import torch
+
+import oracle
+from mixture_experts_ffn_token_b200 import abi
+from mixture_experts_ffn_token_b200.workloads import bf16_bits, make_inputs
+
+# Tolerances, stated once.  Routing and indexing are compared bit-exactly.
+FFN_TOL = 2e-2      # max |gpu - ref| <= FFN_TOL * max |ref|  (bf16 output, fp32 accumulation)
+WEIGHT_RTOL = 1e-5  # router weights (fp32) relative to the fp64 oracle
+WEIGHT_ATOL = 1e-30
+
+
+def to_dev(inp, device="cuda"):
+    return {k: (None if v is None else v.to(device)) for k, v in inp.items()}
+
+
+def oracle_route(wl, inp):
+    logits = inp["logits"].cpu().numpy()
+    if wl.router == "softmax_topk":
+        idx, w = oracle.route_softmax_topk(logits, wl.num_experts, wl.top_k)
+        return idx, w, np.zeros((idx.shape[0], 0))
+    bias = None if inp["expert_bias"] is None else inp["expert_bias"].cpu().numpy()
+    return oracle.route_sigmoid_sink(logits, wl.num_experts, wl.num_sink, wl.top_k, bias, wl.route_scale,
+                                     float(inp["global_scale"][0]))
+
+
+def oracle_ffn(wl, inp, idx, w, tokens=None):
+    return oracle.expert_ffn(bf16_bits(inp["x"]), idx, w, bf16_bits(inp["W_gu"]), bf16_bits(inp["W_d"]),
+                             bf16_bits(inp["b_gu"]), bf16_bits(inp["b_d"]), wl.gate_up_format, wl.activation,
+                             wl.alpha, wl.limit, tokens=tokens)
+
+
+class GpuRun:
+    """One moe_forward call with every output kept for comparison."""
+
+    def __init__(self, wl, d, out_guard=0):
+        T, H, k, S = wl.num_tokens, wl.hidden_dim, wl.top_k, wl.num_sink
+        self.cfg = abi.make_config(wl)
+        self.ws = torch.empty(abi.moe_workspace_size(self.cfg), dtype=torch.uint8, device="cuda")
+        self.out_full = torch.full((T * H + out_guard,), -7.0, dtype=torch.bfloat16, device="cuda")
+        self.out = self.out_full[:T * H].view(T, H)
+        self.idx = torch.full((T, k), -1, dtype=torch.int32, device="cuda")
+        self.w = torch.full((T, k), -1.0, dtype=torch.float32, device="cuda")
+        self.sink = torch.full((T, S), -1.0, dtype=torch.float32, device="cuda") if S > 0 else None
+        abi.moe_forward(self.cfg, d["x"], d["logits"], d["W_gu"], d["W_d"], self.out, self.ws, gate_up_b=d["b_gu"],
+                        down_b=d["b_d"], expert_bias=d["expert_bias"], global_scale=d["global_scale"],
+                        expert_indices_out=self.idx, expert_weights_out=self.w, sink_weights_out=self.sink)
+        torch.cuda.synchronize()
+        self.status = abi.moe_device_status(self.ws)
+
+
+def ffn_error(got, ref):
+    """max |got - ref| / max |ref|."""
+    got = np.asarray(got, dtype=np.float64)
+    scale = np.abs(ref).max()
+    return float(np.abs(got - ref).max() / max(scale, 1e-30))
+
+
+def check_weights(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    err = np.abs(got - ref)
+    assert (err <= WEIGHT_RTOL * np.abs(ref) + WEIGHT_ATOL).all(), float((err / np.maximum(np.abs(ref), 1e-30)).max())
+
+
+def run_and_check(wl, seed=0, device_inputs=False, sample_tokens=None, out_guard=64):
+    """moe_forward against the oracle: routing bit-exact, weights 1e-5, output FFN_TOL."""
+    inp = make_inputs(wl, seed, device="cuda" if device_inputs else "cpu")
+    d = to_dev(inp)
+    run = GpuRun(wl, d, out_guard=out_guard)
+    assert run.status == 0, f"device status {run.status:#x}"
+    idx_ref, w_ref, s_ref = oracle_route(wl, inp)
+    idx = run.idx.cpu().numpy()
+    assert np.array_equal(idx, idx_ref), f"{int((idx != idx_ref).sum())} routing mismatches"
+    check_weights(run.w.cpu().numpy(), w_ref)
+    if wl.num_sink > 0:
+        check_weights(run.sink.cpu().numpy(), s_ref)
+    tokens = None if sample_tokens is None else np.asarray(sample_tokens, dtype=np.int64)
+    ref = oracle_ffn(wl, inp, idx_ref, w_ref, tokens)
+    got = run.out.float().cpu().numpy()
+    if tokens is not None:
+        got = got[tokens]
+    err = ffn_error(got, ref)
+    assert err <= FFN_TOL, f"ffn error {err:.3e} > {FFN_TOL}"
+    if out_guard:
+        guard = run.out_full[wl.num_tokens * wl.hidden_dim:].float()
+        assert (guard == -7.0).all(), "output guard overwritten"
+    return run, err

@@ -1,0 +1,223 @@
+"""CUDA path against the fp64 oracle, element by element, on seeded inputs.
+
+Bars (stated in gpu_helpers): expert indices, CSR offsets and permutation
+bit-exact; router weights within 1e-5 relative; layer output within
+2e-2 * max|ref| (bf16 output, fp32 accumulation).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import FFN_TOL, GpuRun, check_weights, ffn_error, oracle_ffn, oracle_route, run_and_check, to_dev
+from mixture_experts_ffn_token_b200 import abi
+from mixture_experts_ffn_token_b200.workloads import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+# Scaled-down versions of every named workload: several tiles in M and N,
+# ragged row pieces, K and N tails (hidden 328 and moe_dim 200/136 are not
+# multiples of the 64/128/256 tile edges).
+SMALL = {
+    "tiny": WORKLOADS["tiny"],
+    "mixtral_small": WORKLOADS["mixtral"].replace(num_tokens=256, hidden_dim=512, moe_dim=384,
+                                                   logits_std=0.02 * math.sqrt(512)),
+    "gptoss_small": WORKLOADS["gptoss"].replace(num_tokens=96, hidden_dim=328, num_experts=16, moe_dim=200),
+    "sink_small": WORKLOADS["sink"].replace(num_tokens=300, hidden_dim=256, num_experts=32, moe_dim=136),
+    "decode_small": WORKLOADS["decode"].replace(num_tokens=8, hidden_dim=512, num_experts=16, moe_dim=192),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_forward_small(name):
+    run_and_check(SMALL[name], seed=0)
+
+
+@pytest.mark.parametrize("seed", [1, 2])
+def test_forward_tiny_seeds(seed):
+    run_and_check(WORKLOADS["tiny"], seed=seed)
+
+
+@pytest.mark.parametrize("variant", [
+    dict(num_tokens=1), dict(top_k=1), dict(num_tokens=3, top_k=8), dict(num_experts=37, logits_std=1.0),
+    dict(num_experts=64, num_tokens=4),                         # most experts empty
+    dict(gate_up_format="interleaved"), dict(activation="gelu_tanh"),
+    dict(activation="silu", limit=0.05),                        # clamps active on N(0,.) projections
+    dict(activation="swigluoai", alpha=1.702, limit=0.05, has_bias=True),
+    dict(num_tokens=200, hidden_dim=8, moe_dim=8),              # single partial K block, tiny N
+])
+def test_forward_edge_cases(variant):
+    run_and_check(WORKLOADS["tiny"].replace(**variant), seed=3)
+
+
+def test_all_tokens_on_one_expert():
+    wl = WORKLOADS["tiny"].replace(num_tokens=150, top_k=2)
+    inp = make_inputs(wl, 4)
+    inp["logits"][:, 5] += 100.0        # expert 5 first for every token; every other segment is short or empty
+    d = to_dev(inp)
+    run = GpuRun(wl, d)
+    idx_ref, w_ref, _ = oracle_route(wl, inp)
+    assert (idx_ref[:, 0] == 5).all()
+    assert np.array_equal(run.idx.cpu().numpy(), idx_ref)
+    ref = oracle_ffn(wl, inp, idx_ref, w_ref)
+    assert ffn_error(run.out.float().cpu().numpy(), ref) <= FFN_TOL
+
+
+def test_bf16_logits_and_wide_rows():
+    wl = WORKLOADS["sink"].replace(num_tokens=77, hidden_dim=64, num_experts=20, moe_dim=64)
+    inp = make_inputs(wl, 5)
+    T, C = inp["logits"].shape
+    wide = torch.full((T, C + 9), float("nan"))
+    wide[:, :C] = inp["logits"].to(torch.bfloat16).float()
+    cfg = abi.make_config(wl, logits_dtype=torch.bfloat16, logits_row_stride=C + 9)
+    lg = wide.to(torch.bfloat16).cuda()
+    idx = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, wl.top_k), dtype=torch.float32, device="cuda")
+    sw = torch.empty((T, wl.num_sink), dtype=torch.float32, device="cuda")
+    abi.moe_route(cfg, lg, idx, w, sw, inp["expert_bias"].cuda(), inp["global_scale"].cuda())
+    bits = wide.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    i_ref, w_ref, s_ref = oracle.route_sigmoid_sink(bits, wl.num_experts, wl.num_sink, wl.top_k,
+                                                    inp["expert_bias"].numpy(), wl.route_scale, 1.0)
+    assert np.array_equal(idx.cpu().numpy(), i_ref)
+    check_weights(w.cpu().numpy(), w_ref)
+    check_weights(sw.cpu().numpy(), s_ref)
+
+
+@pytest.mark.parametrize("E,k,logits_dtype", [(8, 2, torch.float32), (37, 5, torch.bfloat16), (128, 4, torch.float32),
+                                             (1024, 32, torch.float32), (1, 1, torch.float32)])
+def test_softmax_router(E, k, logits_dtype):
+    T = 513
+    g = torch.Generator().manual_seed(E * 7 + k)
+    logits = (torch.randn(T, E, generator=g) * 2).to(logits_dtype)
+    logits[7, :] = 0.5                    # all ties: lowest indices, in order
+    wl = WORKLOADS["tiny"].replace(num_experts=E, top_k=k, num_tokens=T)
+    cfg = abi.make_config(wl, logits_dtype=logits_dtype)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    abi.moe_route(cfg, logits.cuda(), idx, w)
+    host = logits.float().numpy() if logits_dtype == torch.float32 else \
+        logits.view(torch.int16).numpy().view(np.uint16)
+    i_ref, w_ref = oracle.route_softmax_topk(host, E, k)
+    assert np.array_equal(idx.cpu().numpy(), i_ref)
+    assert idx[7].tolist() == list(range(k))
+    check_weights(w.cpu().numpy(), w_ref)
+
+
+def test_sink_router_extremes():
+    wl = WORKLOADS["sink"].replace(num_tokens=64, num_experts=40, top_k=6, num_sink=2)
+    g = torch.Generator().manual_seed(9)
+    logits = torch.randn(64, 42, generator=g) * 30          # sigmoids saturate and underflow
+    logits[3] = -850.0                                     # every sigmoid underflows: log-space weights
+    bias = (torch.rand(40, generator=g) * 0.2 - 0.1)
+    cfg = abi.make_config(wl)
+    idx = torch.empty((64, 6), dtype=torch.int32, device="cuda")
+    w = torch.empty((64, 6), dtype=torch.float32, device="cuda")
+    sw = torch.empty((64, 2), dtype=torch.float32, device="cuda")
+    gs = torch.tensor([0.75], device="cuda")
+    abi.moe_route(cfg, logits.cuda(), idx, w, sw, bias.cuda(), gs)
+    i_ref, w_ref, s_ref = oracle.route_sigmoid_sink(logits.numpy(), 40, 2, 6, bias.numpy(), wl.route_scale, 0.75)
+    assert np.array_equal(idx.cpu().numpy(), i_ref)
+    check_weights(w.cpu().numpy(), w_ref)
+    check_weights(sw.cpu().numpy(), s_ref)
+    tot = w.double().sum(1) + sw.double().sum(1)
+    assert torch.allclose(tot.cpu(), torch.full((64,), 2.5 * 0.75, dtype=torch.float64), rtol=1e-6)
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 1, 1), (1000, 16, 4), (4096, 128, 6), (7, 1024, 3), (50000, 8, 2)])
+def test_create_indices(T, E, k):
+    g = torch.Generator().manual_seed(T + E)
+    idx = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32) if T < 5000 else \
+        torch.argsort(torch.rand(T, E, generator=g), dim=1)[:, :k].to(torch.int32)
+    wl = WORKLOADS["tiny"].replace(num_tokens=T, num_experts=E, top_k=k)
+    cfg = abi.make_config(wl)
+    ws = torch.empty(abi.moe_workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    abi.moe_create_indices(cfg, idx.cuda(), off, perm, inv, ws)
+    counts, o_ref, p_ref, i_ref = oracle.create_indices(idx.numpy(), E)
+    assert np.array_equal(off.cpu().numpy(), o_ref)
+    assert np.array_equal(perm.cpu().numpy(), p_ref)
+    assert np.array_equal(inv.cpu().numpy(), i_ref)
+    assert abi.moe_device_status(ws) == 0
+
+
+def test_create_indices_flags_bad_expert():
+    wl = WORKLOADS["tiny"].replace(num_tokens=10, num_experts=8, top_k=2)
+    cfg = abi.make_config(wl)
+    idx = torch.randint(0, 8, (10, 2), dtype=torch.int32)
+    idx[4, 1] = 8
+    idx[6, 0] = -3
+    ws = torch.empty(abi.moe_workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    off = torch.empty(9, dtype=torch.int32, device="cuda")
+    perm = torch.full((20,), -1, dtype=torch.int32, device="cuda")
+    abi.moe_create_indices(cfg, idx.cuda(), off, perm, None, ws)
+    assert abi.moe_device_status(ws) & abi.DEVICE_ERR_EXPERT_INDEX
+    assert int(off[-1]) == 18                      # the two bad slots are left out
+
+
+def test_stages_compose_to_forward():
+    """moe_route -> moe_create_indices -> moe_grouped_ffn equals moe_forward bit for bit."""
+    wl = SMALL["gptoss_small"]
+    inp = make_inputs(wl, 6)
+    d = to_dev(inp)
+    run = GpuRun(wl, d)
+    T, k, E = wl.num_tokens, wl.top_k, wl.num_experts
+    cfg = run.cfg
+    ws = torch.empty_like(run.ws)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    abi.moe_route(cfg, d["logits"], idx, w)
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    abi.moe_create_indices(cfg, idx, off, perm, None, ws)
+    out = torch.empty((T, wl.hidden_dim), dtype=torch.bfloat16, device="cuda")
+    abi.moe_grouped_ffn(cfg, d["x"], d["W_gu"], d["b_gu"], d["W_d"], d["b_d"], off, perm, w, out, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, run.idx) and torch.equal(w, run.w)
+    assert torch.equal(out, run.out)
+    again = GpuRun(wl, d)
+    assert torch.equal(again.out, run.out)         # deterministic
+
+
+def test_grouped_ffn_rejects_inconsistent_csr():
+    wl = WORKLOADS["tiny"]
+    inp = make_inputs(wl, 7)
+    d = to_dev(inp)
+    cfg = abi.make_config(wl)
+    ws = torch.empty(abi.moe_workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    off = torch.tensor([0, 10, 5, 40, 60, 80, 100, 120, 128], dtype=torch.int32, device="cuda")  # not monotone
+    perm = torch.arange(128, dtype=torch.int32, device="cuda")
+    w = torch.ones((64, 2), dtype=torch.float32, device="cuda")
+    out = torch.empty((64, 256), dtype=torch.bfloat16, device="cuda")
+    abi.moe_grouped_ffn(cfg, d["x"], d["W_gu"], None, d["W_d"], None, off, perm, w, out, ws)
+    assert abi.moe_device_status(ws) & abi.DEVICE_ERR_CSR
+
+
+def test_zero_tokens():
+    wl = WORKLOADS["tiny"].replace(num_tokens=0)
+    cfg = abi.make_config(wl)
+    ws = torch.zeros(abi.moe_workspace_size(cfg) + 256, dtype=torch.uint8, device="cuda")
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    lg = torch.empty((0, 8), dtype=torch.float32, device="cuda")
+    W = make_inputs(WORKLOADS["tiny"], 0, device="cuda")
+    out = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    abi.moe_forward(cfg, x, lg, W["W_gu"], W["W_d"], out, ws)
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------- full size
+FULL_SAMPLE = 12
+
+
+@pytest.mark.parametrize("name", ["mixtral", "gptoss", "sink", "decode"])
+def test_forward_full_size_sampled(name):
+    """Full-size workloads in the benchmark's launch configuration; routing and
+    CSR are compared for every token, the layer output on sampled tokens."""
+    wl = WORKLOADS[name]
+    T = wl.num_tokens
+    rng = np.random.default_rng(123)
+    sample = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=min(T, FULL_SAMPLE), replace=False)]))
+    run_and_check(wl, seed=0, device_inputs=True, sample_tokens=sample)
