@@ -21,9 +21,7 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import torch
@@ -39,13 +37,6 @@ UNIT = "tokens/s"
 DEFAULT_CONFIG = "mixtral"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = {
-    "gemm_gate_up": "mixture_experts_ffn_token_b200/csrc/grouped_gemm.cu",
-    "gemm_down": "mixture_experts_ffn_token_b200/csrc/grouped_gemm.cu",
-    "router": "mixture_experts_ffn_token_b200/csrc/router.cu",
-    "gather": "mixture_experts_ffn_token_b200/csrc/csr.cu",
-    "combine": "mixture_experts_ffn_token_b200/csrc/csr.cu",
-}
 
 
 # ------------------------------------------------------------------ helpers
@@ -54,6 +45,20 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def max_over_ranks(x, dist_mod, device):
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if dist_mod is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, tokens_per_rank, ms_per_step):
+    """Whole-job tokens/s: every rank runs its own batch of tokens_per_rank."""
+    return world * tokens_per_rank / (ms_per_step / 1000.0)
 
 
 def load_peaks():
@@ -80,89 +85,89 @@ def touched_expert_bytes(wl, idx):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+    """SM clocks and clock-event (throttle) reasons sampled every few
+    milliseconds by a host thread through NVML (the counters nvidia-smi
+    reads) while the timed region runs."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, device_index):
-        self.proc = None
-        self.path = None
+    def __init__(self, device_index, period_s=0.005):
+        import threading
+        self.period = period_s
+        self.samples = []
+        self.error = None
+        self.stop_evt = threading.Event()
+        self.thread = None
+        self.nvml = None
         try:
+            import pynvml
+            pynvml.nvmlInit()
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
-            target = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
-        except Exception:
-            target = []
-        self.cmd = ["nvidia-smi", *target, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                    "-lms", "100"]
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.nvml = pynvml
+        except Exception as exc:  # no NVML: report it instead of guessing
+            self.error = f"nvml unavailable: {exc}"
+
+    def _run(self):
+        p = self.nvml
+        while not self.stop_evt.is_set():
+            try:
+                mhz = p.nvmlDeviceGetClockInfo(self.handle, p.NVML_CLOCK_SM)
+                mask = p.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                watts = p.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                self.samples.append((mhz, mask, watts))
+            except Exception as exc:
+                self.error = str(exc)
+                return
+            time.sleep(self.period)
 
     def __enter__(self):
-        try:
-            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
-            self.fh = os.fdopen(fd, "w")
-            self.proc = subprocess.Popen(self.cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
-            time.sleep(0.25)
-        except Exception:
-            self.proc = None
+        if self.nvml is not None:
+            import threading
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            time.sleep(0.15)
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.fh.close()
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
 
     def summary(self):
-        if self.proc is None or self.path is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 8:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-
-        def num(s):
-            try:
-                return float(s)
-            except ValueError:
-                return None
-        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
-        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows),
-                "power_w_max": max((num(r[2]) or 0.0) for r in rows)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "no samples"]}
+        p = self.nvml
+        reasons = sorted({name for name, attr in self.REASONS for (_, mask, _) in self.samples
+                          if mask & getattr(p, attr)})
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml",
+                "power_w_max": max(s[2] for s in self.samples)}
 
 
-def kernel_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it
-    was taken from the current source of that kernel (else None)."""
+def kernel_traffic(workload, kernel):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary (profiles/traffic.json), if it was captured from the kernel's
+    current source; otherwise None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        data = json.load(f)
-    ent = data.get(kernel)
+        ent = json.load(f).get(workload, {}).get(kernel)
     if not ent:
         return None
-    src = os.path.join(ROOT, KERNEL_SOURCES.get(kernel, ""))
-    if not os.path.exists(src):
+    src = os.path.join(ROOT, ent.get("source", ""))
+    if not os.path.isfile(src):
         return None
     with open(src, "rb") as f:
         digest = hashlib.sha256(f.read()).hexdigest()[:16]
     if ent.get("source_sha256_16") != digest:
         return None
-    return ent.get("bytes_per_launch_full_size")
+    return ent.get("bytes_per_launch")
 
 
 # ---------------------------------------------------------------- oracle arm
@@ -194,21 +199,34 @@ def oracle_sample_rate(wl, inp_host, n_tokens, seed=0):
 
 
 def host_inputs_for_oracle(wl, seed, device):
-    from mixture_experts_ffn_token_b200.workloads import bf16_bits
     inp = make_inputs(wl, seed, device=device)
+    return inp, host_copy_for_oracle(inp)
+
+
+def host_copy_for_oracle(inp):
+    from mixture_experts_ffn_token_b200.workloads import bf16_bits
     host = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
     host["x_bits"] = bf16_bits(host["x"])
     host["W_gu_bits"] = bf16_bits(host["W_gu"])
     host["W_d_bits"] = bf16_bits(host["W_d"])
     host["b_gu_bits"] = bf16_bits(host["b_gu"])
     host["b_d_bits"] = bf16_bits(host["b_d"])
-    return inp, host
+    return host
 
 
 def calibrated_sample(wl, host, seconds):
-    """Smallest sample that takes about `seconds` of oracle time (>= 1 token)."""
-    rate, dt, thr = oracle_sample_rate(wl, host, 1, seed=99)
-    n = max(1, min(wl.num_tokens, int(rate * seconds)))
+    """A token sample that takes about `seconds` of oracle time (>= 1 token).
+    Two probes: the oracle parallelises over the slots of one expert, so its
+    rate grows with the sample until the host cores are busy."""
+    n = 1
+    rate, thr = 0.0, 1
+    for _ in range(3):
+        rate, dt, thr = oracle_sample_rate(wl, host, n, seed=99)
+        target = max(1, min(wl.num_tokens, int(rate * seconds)))
+        if dt > 0.25 * seconds or target <= n:
+            n = target
+            break
+        n = min(target, max(2 * n, target // 4))
     return n, rate, thr
 
 
@@ -254,6 +272,59 @@ def config_block(wl, world):
 
 
 # ------------------------------------------------------------------ GPU arm
+def run_e2e(args, cfg, inp, kw, ws, stream, dist):
+    """K steps of moe_forward fed from, and returning to, pinned host memory.
+    Returns the device time (max over ranks) of the whole region in ms."""
+    T, H = inp["x"].shape
+    x_h = inp["x"].cpu().pin_memory()
+    lg_h = inp["logits"].cpu().pin_memory()
+    out_h = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_d = [torch.empty_like(inp["x"]) for _ in range(2)]
+    lg_d = [torch.empty_like(inp["logits"]) for _ in range(2)]
+    out_d = [torch.empty((T, H), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def region(steps):
+        in_ready = [torch.cuda.Event() for _ in range(steps)]
+        fwd_done = [torch.cuda.Event() for _ in range(steps)]
+        out_done = [torch.cuda.Event() for _ in range(steps)]
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        h2d.wait_event(start)
+        d2h.wait_event(start)
+        for i in range(steps):
+            b = i % 2
+            with torch.cuda.stream(h2d):
+                if i >= 2:
+                    h2d.wait_event(fwd_done[i - 2])        # buffer b no longer read by step i-2
+                x_d[b].copy_(x_h, non_blocking=True)
+                lg_d[b].copy_(lg_h, non_blocking=True)
+                in_ready[i].record(h2d)
+            stream.wait_event(in_ready[i])
+            if i >= 2:
+                stream.wait_event(out_done[i - 2])         # out_d[b] copied out by step i-2
+            abi.moe_forward(cfg, x_d[b], lg_d[b], inp["W_gu"], inp["W_d"], out_d[b], ws, stream=stream, **kw)
+            fwd_done[i].record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(fwd_done[i])
+                out_h[b].copy_(out_d[b], non_blocking=True)
+                out_done[i].record(d2h)
+        stream.wait_event(out_done[steps - 1])
+        stream.wait_event(out_done[steps - 2] if steps > 1 else out_done[steps - 1])
+        stop.record(stream)
+        torch.cuda.synchronize()
+        return start.elapsed_time(stop)
+
+    region(max(2, args.warmup))
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms = region(args.steps)
+    if not torch.equal(out_h[(args.steps - 1) % 2], out_d[(args.steps - 1) % 2].cpu()):
+        raise RuntimeError("e2e: host copy of the output differs from the device result")
+    return max_over_ranks(ms, dist, "cuda")
+
+
 def run_gpu(args, wl):
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -297,6 +368,9 @@ def run_gpu(args, wl):
     # events on the launching stream, read after the region
     n_ev = abi.NUM_STAGE_EVENTS
     ev_sets = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    for evs in ev_sets:          # create the CUDA events outside the timed region
+        for ev in evs:
+            ev.record(stream)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -325,42 +399,18 @@ def run_gpu(args, wl):
     status = abi.moe_device_status(ws)
     if status != 0:
         raise RuntimeError(f"device status {status:#x} after the timed region")
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, "cuda")
     ms_per_step = elapsed_ms / args.steps
-    value = world * T / (ms_per_step / 1000.0)
+    value = job_throughput(world, T, ms_per_step)
 
-    # ---------------- e2e: host buffers, H2D inputs + D2H output inside the region
-    x_h = inp["x"].cpu().pin_memory()
-    lg_h = inp["logits"].cpu().pin_memory()
-    out_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
-    x_d = torch.empty_like(inp["x"])
-    lg_d = torch.empty_like(inp["logits"])
-    for _ in range(max(1, args.warmup // 2)):
-        x_d.copy_(x_h, non_blocking=True)
-        lg_d.copy_(lg_h, non_blocking=True)
-        abi.moe_forward(cfg, x_d, lg_d, inp["W_gu"], inp["W_d"], out, ws, **kw)
-        out_h.copy_(out, non_blocking=True)
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_start.record(stream)
-    for _ in range(args.steps):
-        x_d.copy_(x_h, non_blocking=True)
-        lg_d.copy_(lg_h, non_blocking=True)
-        abi.moe_forward(cfg, x_d, lg_d, inp["W_gu"], inp["W_d"], out, ws, **kw)
-        out_h.copy_(out, non_blocking=True)
-    e_stop.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e_start.elapsed_time(e_stop)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * T / (e2e_ms / args.steps / 1000.0)
+    # ---------------- e2e: host buffers; every step copies its inputs host->device
+    # from pinned memory and its output device->host inside the timed region.
+    # Copies run on their own streams, double-buffered, so step i's copies
+    # overlap the compute of its neighbours.
+    e2e_ms = run_e2e(args, cfg, inp, kw, ws, stream, dist)
+    e2e_value = job_throughput(world, T, e2e_ms / args.steps)
+    x_h_bytes = inp["x"].numel() * 2 + inp["logits"].numel() * 4
+    out_bytes = T * H * 2
 
     # ---------------- roofline of the dominant kernel
     names = abi.STAGE_NAMES
@@ -370,16 +420,21 @@ def run_gpu(args, wl):
     down_flops = 2 * T * k * H * wl.moe_dim
     dom = max(range(len(names)), key=lambda i: stage_ms[i])
     dom_name = names[dom]
-    sustained = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    clock_summary = clocks.summary()
+    # a GEMM timed while the power cap held the clocks down is compared with
+    # the sustained bf16 figure, otherwise with the burst figure
+    capped = "sw_power_cap" in clock_summary.get("reasons", [])
+    bf16_peak = peaks.get("bf16_tflops_sustained" if capped else "bf16_tflops", peaks.get("bf16_tflops"))
+    bf16_kind = "sustained" if capped else "burst"
     if dom_name in ("gemm_gate_up", "gemm_down"):
         kflops = gate_up_flops if dom_name == "gemm_gate_up" else down_flops
         kbytes = (2 if dom_name == "gemm_gate_up" else 1) * used * H * wl.moe_dim * 2
-        t_flop = kflops / (sustained * 1e12)
+        t_flop = kflops / (bf16_peak * 1e12)
         t_byte = kbytes / (peaks["hbm_gbs"] * 1e9)
         if t_flop >= t_byte:
             achieved = kflops / (stage_ms[dom] / 1e3) / 1e12
-            roof = {"bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
-                    "peak_kind": f"{peak_kind} bf16 sustained"}
+            roof = {"bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
+                    "peak_kind": f"{peak_kind} bf16 {bf16_kind}"}
         else:
             achieved = kbytes / (stage_ms[dom] / 1e3) / 1e9
             roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -391,7 +446,7 @@ def run_gpu(args, wl):
                 "peak_kind": f"{peak_kind} hbm copy"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["kernel"] = dom_name
-    roof["traffic"] = kernel_traffic(dom_name)
+    roof["traffic"] = kernel_traffic(wl.name, dom_name)
     roof["kernel_ms"] = stage_ms[dom]
 
     line = {
@@ -404,14 +459,13 @@ def run_gpu(args, wl):
         "experts_touched": used,
         "stages_ms": {n: round(v, 5) for n, v in zip(names, stage_ms)},
         "roofline": roof,
-        "e2e": {"value": e2e_value, "unit": UNIT,
-                "h2d_bytes_per_step": x_h.numel() * 2 + lg_h.numel() * 4,
-                "d2h_bytes_per_step": out_h.numel() * 2},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x_h_bytes,
+                "d2h_bytes_per_step": out_bytes},
         "gpu_launches": 8 * args.steps,
-        "clocks": clocks.summary(),
+        "clocks": clock_summary,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl)
+        line["cpu_baseline"] = cpu_baseline(wl, inp)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -420,8 +474,8 @@ def run_gpu(args, wl):
     return 0
 
 
-def cpu_baseline(wl):
-    _, host = host_inputs_for_oracle(wl, 0, "cuda")
+def cpu_baseline(wl, inp):
+    host = host_copy_for_oracle(inp)
     n, _, _ = calibrated_sample(wl, host, 15.0)
     rate, dt, threads = oracle_sample_rate(wl, host, n, seed=7)
     return {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",

@@ -174,6 +174,11 @@ def moe_forward_timed(cfg, events, x, logits, gate_up_w, down_w, out, workspace,
                       expert_bias=None, global_scale=None, expert_indices_out=None, expert_weights_out=None,
                       sink_weights_out=None, stream=None):
     """moe_forward recording torch.cuda.Event objects `events` (9) between stages."""
+    if len(events) != NUM_STAGE_EVENTS:
+        raise ValueError(f"moe_forward_timed needs {NUM_STAGE_EVENTS} events")
+    for ev in events:
+        if ev.cuda_event == 0:      # torch creates the CUDA event on its first record
+            ev.record(stream)
     arr = (ctypes.c_void_p * NUM_STAGE_EVENTS)(*[ev.cuda_event for ev in events])
     _check(load_library().moe_forward_timed(ctypes.byref(cfg), _p(x), _p(logits), _p(expert_bias),
                                             _p(global_scale), _p(gate_up_w), _p(gate_up_b), _p(down_w), _p(down_b),

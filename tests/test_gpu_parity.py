@@ -182,6 +182,21 @@ def test_stages_compose_to_forward():
     assert torch.equal(again.out, run.out)         # deterministic
 
 
+def test_forward_timed_matches_forward():
+    wl = SMALL["sink_small"]
+    d = to_dev(make_inputs(wl, 8))
+    run = GpuRun(wl, d)
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(abi.NUM_STAGE_EVENTS)]
+    out = torch.empty_like(run.out)
+    sink = torch.empty_like(run.sink)
+    abi.moe_forward_timed(run.cfg, events, d["x"], d["logits"], d["W_gu"], d["W_d"], out, run.ws,
+                          expert_bias=d["expert_bias"], global_scale=d["global_scale"], sink_weights_out=sink)
+    torch.cuda.synchronize()
+    assert torch.equal(out, run.out) and torch.equal(sink, run.sink)
+    times = [events[i].elapsed_time(events[i + 1]) for i in range(abi.NUM_STAGE_EVENTS - 1)]
+    assert all(t >= 0 for t in times) and sum(times) > 0
+
+
 def test_grouped_ffn_rejects_inconsistent_csr():
     wl = WORKLOADS["tiny"]
     inp = make_inputs(wl, 7)
