@@ -207,6 +207,36 @@ moe_status_t moe_forward_timed(const moe_config_t* cfg, const void* x, const voi
  * (other bits are reported through *device_status only). */
 moe_status_t moe_device_status(const void* workspace, int32_t* device_status, moe_stream_t stream);
 
+/* moe_create_indices without a workspace.  This entry point has no
+ * counterpart on the documentation pages; it exists for callers that cannot
+ * allocate device memory at the point where they build the routing: code
+ * embedded in a host runtime that owns all device memory through its own pool
+ * (for instance a serving engine that reserves almost all of HBM for its
+ * caches and gives plugins no allocator), and latency-critical paths where
+ * the implicit synchronisation of cudaMalloc/cudaFree is not acceptable.
+ *
+ * It computes exactly what moe_create_indices computes (same arguments
+ * without workspace/workspace_bytes), with its scratch -- the device status
+ * word and the per-chunk histogram and base tables -- in one file-scope
+ * device array of 524,544 bytes that every GPU loading this library holds
+ * until the process exits.  Capacity: ceil(T*k / 2048) * E <= 65,536 (for
+ * example up to 1,048,576 routed slots with E = 128); larger problems get
+ * MOE_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.  The call itself
+ * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  Every call shares the one array, which keeps
+ * the last call's contents (the status word is cleared at the start of each
+ * call, the tables are rewritten): calls that overlap on the GPU -- on two
+ * streams, or from two threads -- race and give undefined results.  Device
+ * fault bits (MOE_DEVICE_ERR_EXPERT_INDEX) land in the array's status word,
+ * which no entry point reads back; out-of-range indices are skipped as in
+ * moe_create_indices. */
+moe_status_t moe_create_indices_noalloc(const moe_config_t* cfg, const int32_t* expert_indices,
+                                        int32_t* expert_offsets, int32_t* permutation, int32_t* inverse,
+                                        moe_stream_t stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -31,7 +31,7 @@ NUM_STAGE_EVENTS = 9
 STAGE_NAMES = ("router", "csr_count", "csr_scan", "csr_scatter", "gather", "gemm_gate_up", "gemm_down", "combine")
 
 EXPORTED = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_create_indices", "moe_grouped_ffn",
-            "moe_forward", "moe_forward_timed", "moe_device_status")
+            "moe_forward", "moe_forward_timed", "moe_device_status", "moe_create_indices_noalloc")
 
 
 class MoEConfig(ctypes.Structure):
@@ -89,6 +89,8 @@ def load_library():
     lib.moe_forward_timed.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
     lib.moe_device_status.restype = ctypes.c_int
     lib.moe_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
+    lib.moe_create_indices_noalloc.restype = ctypes.c_int
+    lib.moe_create_indices_noalloc.argtypes = [cfgp, vp, vp, vp, vp, vp]
     _lib = lib
     return lib
 
@@ -151,6 +153,14 @@ def moe_create_indices(cfg, expert_indices, expert_offsets, permutation, inverse
     _check(load_library().moe_create_indices(ctypes.byref(cfg), _p(expert_indices), _p(expert_offsets),
                                              _p(permutation), _p(inverse), _p(workspace), workspace.numel(),
                                              _stream(stream)), "moe_create_indices")
+
+
+def moe_create_indices_noalloc(cfg, expert_indices, expert_offsets, permutation, inverse=None, stream=None):
+    """moe_create_indices with its scratch in the library's fixed device array
+    (for callers that cannot allocate a workspace)."""
+    _check(load_library().moe_create_indices_noalloc(ctypes.byref(cfg), _p(expert_indices), _p(expert_offsets),
+                                                     _p(permutation), _p(inverse), _stream(stream)),
+           "moe_create_indices_noalloc")
 
 
 def moe_grouped_ffn(cfg, x, gate_up_w, gate_up_b, down_w, down_b, expert_offsets, permutation, expert_weights,

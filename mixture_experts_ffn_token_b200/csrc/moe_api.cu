@@ -379,3 +379,66 @@ moe_status_t moe_device_status(const void* workspace, int32_t* device_status, mo
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// moe_create_indices_noalloc: the same CSR build, with its scratch (the
+// device status word and the per-chunk histogram and base tables) in one
+// fixed-size array in device memory instead of a caller workspace.
+namespace {
+
+// Capacity: (number of 2048-slot chunks) x (experts) cells.  With 128
+// experts that is up to 1,048,576 routed slots; with 1024 experts, 131,072.
+constexpr size_t kNoAllocMaxCells = 65536;
+constexpr size_t kNoAllocHeaderBytes = 256;  // the device status word lives here
+constexpr size_t kNoAllocBytes = kNoAllocHeaderBytes + 2 * kNoAllocMaxCells * sizeof(int32_t);  // 512.25 KiB
+
+// Every GPU that loads this library holds this array until the process
+// exits.  Host code must not use its name as an address: the device address
+// comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (with that device current) on its first call.
+moe_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status_t moe_create_indices_noalloc(const moe_config_t* cfg, const int32_t* expert_indices,
+                                                   int32_t* expert_offsets, int32_t* permutation,
+                                                   int32_t* inverse, moe_stream_t stream) {
+  moe_status_t st = validate_config(cfg);
+  if (st != MOE_OK) return st;
+  if (expert_offsets == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  if (cfg->num_tokens > 0 && (expert_indices == nullptr || permutation == nullptr)) return MOE_ERR_INVALID_ARGUMENT;
+  const int64_t R = static_cast<int64_t>(cfg->num_tokens) * cfg->top_k;
+  const size_t cells = static_cast<size_t>(moe::csr_num_chunks(R)) * static_cast<size_t>(cfg->num_experts);
+  if (cells > kNoAllocMaxCells) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  int num_sms = 0;
+  if ((st = current_device(&num_sms)) != MOE_OK) return st;
+  void* base = nullptr;
+  if ((st = noalloc_scratch(&base)) != MOE_OK) return st;
+  WsLayout L = {};
+  L.status = 0;
+  L.chunk_counts = kNoAllocHeaderBytes;
+  L.chunk_base = kNoAllocHeaderBytes + kNoAllocMaxCells * sizeof(int32_t);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // The histogram and base tables are fully rewritten by every call; only the
+  // status word has to start at zero.
+  if (cudaMemsetAsync(base, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  return enqueue_csr(cfg, expert_indices, expert_offsets, permutation, inverse, base, L, s, nullptr);
+}
