@@ -215,19 +215,17 @@ def host_copy_for_oracle(inp):
 
 
 def calibrated_sample(wl, host, seconds):
-    """A token sample that takes about `seconds` of oracle time (>= 1 token).
-    Two probes: the oracle parallelises over the slots of one expert, so its
-    rate grows with the sample until the host cores are busy."""
+    """Grow a token sample until the oracle spends about `seconds` on it
+    (the oracle parallelises over the slots of one expert, so its rate grows
+    with the sample until the host cores are busy).  Returns (tokens, rate,
+    elapsed, threads) of the last, largest measurement."""
     n = 1
-    rate, thr = 0.0, 1
-    for _ in range(3):
+    while True:
         rate, dt, thr = oracle_sample_rate(wl, host, n, seed=99)
-        target = max(1, min(wl.num_tokens, int(rate * seconds)))
-        if dt > 0.25 * seconds or target <= n:
-            n = target
-            break
-        n = min(target, max(2 * n, target // 4))
-    return n, rate, thr
+        if dt >= 0.5 * seconds or n >= wl.num_tokens:
+            return n, rate, dt, thr
+        grow = min(8.0, max(2.0, 0.8 * seconds / max(dt, 1e-6)))
+        n = min(wl.num_tokens, max(n + 1, int(n * grow)))
 
 
 def run_reference(args, wl):
@@ -238,7 +236,7 @@ def run_reference(args, wl):
     _, host = host_inputs_for_oracle(wl, 0, device)
     budget = 150.0  # seconds of oracle time for the whole run
     per_step = budget / max(1, args.steps + args.warmup)
-    n, _, threads = calibrated_sample(wl, host, per_step)
+    n, _, _, threads = calibrated_sample(wl, host, per_step)
     for i in range(args.warmup):
         oracle_sample_rate(wl, host, n, seed=i)
     times = []
@@ -272,6 +270,28 @@ def config_block(wl, world):
 
 
 # ------------------------------------------------------------------ GPU arm
+def timed_steps(step, steps, stream, flush):
+    """Device time in ms of `steps` calls of step() on `stream`; with `flush`,
+    the L2 is overwritten before every step, outside the timed intervals."""
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if flush is None:
+        start.record(stream)
+        for _ in range(steps):
+            step()
+        stop.record(stream)
+        torch.cuda.synchronize()
+        return start.elapsed_time(stop)
+    total = 0.0
+    for _ in range(steps):
+        flush.fill_(1)
+        start.record(stream)
+        step()
+        stop.record(stream)
+        torch.cuda.synchronize()
+        total += start.elapsed_time(stop)
+    return total
+
+
 def run_e2e(args, cfg, inp, kw, ws, stream, dist):
     """K steps of moe_forward fed from, and returning to, pinned host memory.
     Returns the device time (max over ranks) of the whole region in ms."""
@@ -364,37 +384,31 @@ def run_gpu(args, wl):
     if abi.moe_device_status(ws) != 0:
         raise RuntimeError("device status set during warm-up")
 
-    # ---------------- timed region: K steps; every step records its own stage
-    # events on the launching stream, read after the region
-    n_ev = abi.NUM_STAGE_EVENTS
-    ev_sets = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
-    for evs in ev_sets:          # create the CUDA events outside the timed region
-        for ev in evs:
-            ev.record(stream)
+    # ---------------- timed region: K steps of moe_forward between two CUDA
+    # events on the launching stream (max over ranks); L2 flushed between
+    # steps when the inputs would fit in it
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if flush is None:
-            start.record(stream)
-            for i in range(args.steps):
-                step(ev_sets[i])
-            stop.record(stream)
-            torch.cuda.synchronize()
-            elapsed_ms = start.elapsed_time(stop)
-        else:
-            elapsed_ms = 0.0
-            for i in range(args.steps):
-                flush.fill_(1)
-                start.record(stream)
-                step(ev_sets[i])
-                stop.record(stream)
-                torch.cuda.synchronize()
-                elapsed_ms += start.elapsed_time(stop)
+        elapsed_ms = timed_steps(step, args.steps, stream, flush)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
+
+    # ---------------- stage region: the same K steps through moe_forward_timed,
+    # each step recording its own 9 events on the launching stream; per-kernel
+    # durations for the roofline come from here (a timing event between two
+    # kernels stops them overlapping, so the step total above is taken
+    # without them)
+    n_ev = abi.NUM_STAGE_EVENTS
+    ev_sets = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    for evs in ev_sets:          # create the CUDA events outside the region
+        for ev in evs:
+            ev.record(stream)
+    torch.cuda.synchronize()
+    it = iter(ev_sets)
+    timed_steps(lambda: step(next(it)), args.steps, stream, flush)
     stage_ms = [sum(evs[i].elapsed_time(evs[i + 1]) for evs in ev_sets) / args.steps for i in range(n_ev - 1)]
     status = abi.moe_device_status(ws)
     if status != 0:
@@ -476,8 +490,7 @@ def run_gpu(args, wl):
 
 def cpu_baseline(wl, inp):
     host = host_copy_for_oracle(inp)
-    n, _, _ = calibrated_sample(wl, host, 15.0)
-    rate, dt, threads = oracle_sample_rate(wl, host, n, seed=7)
+    n, rate, dt, threads = calibrated_sample(wl, host, 15.0)
     return {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{n} of {wl.num_tokens} tokens (router + expert FFN, fp64), {dt:.1f} s"}
 

@@ -37,6 +37,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "kernels.cuh"
@@ -44,20 +45,30 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;                 // rows per tile (TMEM lanes)
+constexpr int BM = 128;                 // rows per CTA (TMEM lanes)
 constexpr int BN = 256;                 // accumulator columns per tile
 constexpr int BK = 64;                  // K per stage: one 128-byte swizzle row of bf16
 constexpr int UMMA_K = 16;              // K per tcgen05.mma (kind::f16)
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB
 constexpr int B_BOX_BYTES = BK * 64 * 2;        // 8 KB: 64 K rows x 64 N columns
-constexpr int B_BYTES = 4 * B_BOX_BYTES;        // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;             // two BN-column fp32 accumulators
 constexpr int CTRL_BYTES = 256;
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
-constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, /*a_mn_major=*/false, /*b_mn_major=*/true);
+
+// Per-CTA pipeline geometry.  PAIR = 1: one CTA computes a 128 x 256 tile and
+// loads all four 64-column B boxes (48 KB a stage, 4 stages).  PAIR = 2: a
+// cluster of two CTAs computes a 256 x 256 tile with tcgen05 cta_group::2;
+// each CTA loads its 128 rows of A and its 128 columns of B (32 KB a stage,
+// 6 stages), so each SM streams a third less operand data per FLOP.
+template <int PAIR>
+struct Geo {
+  static constexpr int B_BOXES = 4 / PAIR;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BOXES * B_BOX_BYTES;
+  static constexpr int STAGES = PAIR == 1 ? 4 : 6;
+  static constexpr int PIECE = BM * PAIR;  // rows of one tile
+  static constexpr uint32_t IDESC = idesc_bf16_f32(BM * PAIR, BN, /*a_mn_major=*/false, /*b_mn_major=*/true);
+};
 
 constexpr int MODE_GATE_UP_CONCAT = 0;
 constexpr int MODE_GATE_UP_INTERLEAVED = 1;
@@ -81,9 +92,11 @@ struct TileCoord {
   int e, row0, rows, n;
 };
 
-// Tile t -> (expert, first permuted row, valid rows, output column block).
-// s_mt is the exclusive prefix of per-expert 128-row pieces (s_mt[E] = total).
-__device__ __forceinline__ TileCoord decode_tile(int t, int n_tiles, int E, const int* s_mt, const int* s_off) {
+// Tile t -> (expert, first permuted row of the tile, valid rows, output
+// column block).  s_mt is the exclusive prefix of per-expert pieces of
+// `piece` rows (s_mt[E] = total).
+__device__ __forceinline__ TileCoord decode_tile(int t, int n_tiles, int E, const int* s_mt, const int* s_off,
+                                                 int piece) {
   int lo = 0, hi = E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -96,8 +109,8 @@ __device__ __forceinline__ TileCoord decode_tile(int t, int n_tiles, int E, cons
   const int mt = s_mt[lo + 1] - s_mt[lo];
   c.n = local / mt;
   const int m = local - c.n * mt;
-  c.row0 = s_off[lo] + m * BM;
-  c.rows = min(BM, s_off[lo + 1] - c.row0);
+  c.row0 = s_off[lo] + m * piece;
+  c.rows = min(piece, s_off[lo + 1] - c.row0);
   return c;
 }
 
@@ -233,17 +246,18 @@ __device__ __forceinline__ void epilogue_down(const GemmParams& p, const TileCoo
 }
 
 // ------------------------------------------------------------- the kernel
-template <int MODE>
+template <int MODE, int PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                         const GemmParams p) {
+  using G = Geo<PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  uint8_t* ctrl = smem + STAGES * STAGE_BYTES;
+  uint8_t* ctrl = smem + G::STAGES * G::STAGE_BYTES;
   const uint32_t full0 = smem_u32(ctrl);              // STAGES mbarriers
-  const uint32_t empty0 = full0 + 8 * STAGES;         // STAGES mbarriers
-  const uint32_t tfull0 = empty0 + 8 * STAGES;        // 2 mbarriers
+  const uint32_t empty0 = full0 + 8 * G::STAGES;      // STAGES mbarriers
+  const uint32_t tfull0 = empty0 + 8 * G::STAGES;     // 2 mbarriers
   const uint32_t tempty0 = tfull0 + 16;               // 2 mbarriers
   const uint32_t drain_bar = tempty0 + 16;            // 1 mbarrier
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 128);
@@ -254,15 +268,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR == 2 ? cluster_ctarank() : 0u;  // 0 = leader of the pair
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < G::STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, 128);
+      mbar_init(tempty0 + 8 * a, 128 * PAIR);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -272,13 +288,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_map(&mapB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR == 2) {
+      tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) s_off[i] = p.offsets[i];
   __syncthreads();
   if (warp == 0) {
-    // Validate the CSR and build the per-expert prefix of 128-row pieces.
+    // Validate the CSR and build the per-expert prefix of tile pieces.
     const int per = (p.E + 31) / 32;
     const int e0 = min(lane * per, p.E), e1 = min(e0 + per, p.E);
     int local = 0;
@@ -286,7 +307,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int e = e0; e < e1; ++e) {
       const int cnt = s_off[e + 1] - s_off[e];
       if (cnt < 0) bad = true;
-      else local += (cnt + BM - 1) / BM;
+      else local += (cnt + G::PIECE - 1) / G::PIECE;
     }
     int incl = local;
 #pragma unroll
@@ -298,80 +319,107 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int e = e0; e < e1; ++e) {
       s_mt[e] = run;
       const int cnt = s_off[e + 1] - s_off[e];
-      if (cnt > 0) run += (cnt + BM - 1) / BM;
+      if (cnt > 0) run += (cnt + G::PIECE - 1) / G::PIECE;
     }
     if (lane == 31) s_mt[p.E] = incl;
     if (lane == 0 && (s_off[0] != 0 || s_off[p.E] > p.R)) bad = true;
     if (__any_sync(0xffffffffu, bad) && lane == 0) *bad_flag = 1;
   }
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (PAIR == 2) {
+    cluster_sync();  // both CTAs' barriers exist before either signals the other's
+  } else {
+    __syncthreads();
+  }
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
   const bool bad = *bad_flag != 0;
   if (bad && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, MOE_DEVICE_ERR_CSR);
   const int total_tiles = bad ? 0 : s_mt[p.E] * p.n_tiles;
+  const int first_tile = blockIdx.x / PAIR;
+  const int tile_stride = gridDim.x / PAIR;
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
       int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
-        const TileCoord tc = decode_tile(t, p.n_tiles, p.E, s_mt, s_off);
+      for (int t = first_tile; ok && t < total_tiles; t += tile_stride) {
+        const TileCoord tc = decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
+        const int arow = tc.row0 + static_cast<int>(rank) * BM;
         for (int kb = 0; kb < p.num_kb; ++kb) {
-          const int s = it % STAGES;
-          const uint32_t ph = static_cast<uint32_t>(it / STAGES) & 1u;
+          const int s = it % G::STAGES;
+          const uint32_t ph = static_cast<uint32_t>(it / G::STAGES) & 1u;
           if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kTimeoutNs)) {
             ok = false;
             break;
           }
-          const uint32_t sa = sbase + s * STAGE_BYTES;
+          const uint32_t sa = sbase + s * G::STAGE_BYTES;
           const uint32_t sb = sa + A_BYTES;
-          const uint32_t fb = full0 + 8 * s;
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          tma_load_2d(sa, &mapA, fb, kb * BK, tc.row0);
-          if constexpr (MODE == MODE_GATE_UP_CONCAT) {
-            // 4-D view {D, 2 (gate/up), H, E}: two gate boxes then two up boxes.
-            const int c0 = tc.n * 128;
-            tma_load_4d(sb, &mapB, fb, c0, 0, kb * BK, tc.e);
-            tma_load_4d(sb + B_BOX_BYTES, &mapB, fb, c0 + 64, 0, kb * BK, tc.e);
-            tma_load_4d(sb + 2 * B_BOX_BYTES, &mapB, fb, c0, 1, kb * BK, tc.e);
-            tma_load_4d(sb + 3 * B_BOX_BYTES, &mapB, fb, c0 + 64, 1, kb * BK, tc.e);
-          } else {
-            // 3-D view {N, K, E}: four consecutive 64-column boxes.
-            const int c0 = tc.n * BN;
+          // the leader's full barrier counts both CTAs' bytes
+          const uint32_t fb = PAIR == 2 ? map_to_rank(full0 + 8 * s, 0) : full0 + 8 * s;
+          const int kc = kb * BK;
+          if constexpr (PAIR == 1) {
+            mbar_arrive_expect_tx(fb, G::STAGE_BYTES);
+            tma_load_2d(sa, &mapA, fb, kc, arow);
+            if constexpr (MODE == MODE_GATE_UP_CONCAT) {
+              // 4-D view {D, 2 (gate/up), H, E}: two gate boxes then two up boxes.
+              const int c0 = tc.n * 128;
+              tma_load_4d(sb, &mapB, fb, c0, 0, kc, tc.e);
+              tma_load_4d(sb + B_BOX_BYTES, &mapB, fb, c0 + 64, 0, kc, tc.e);
+              tma_load_4d(sb + 2 * B_BOX_BYTES, &mapB, fb, c0, 1, kc, tc.e);
+              tma_load_4d(sb + 3 * B_BOX_BYTES, &mapB, fb, c0 + 64, 1, kc, tc.e);
+            } else {
+              // 3-D view {N, K, E}: four consecutive 64-column boxes.
+              const int c0 = tc.n * BN;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * B_BOX_BYTES, &mapB, fb, c0 + 64 * j, kb * BK, tc.e);
+              for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * B_BOX_BYTES, &mapB, fb, c0 + 64 * j, kc, tc.e);
+            }
+          } else {
+            // The leader expects both CTAs' bytes on its own barrier; each
+            // CTA loads its 128 rows of A and its half of the 256 columns.
+            if (leader) mbar_arrive_expect_tx(full0 + 8 * s, 2 * G::STAGE_BYTES);
+            tma_load_2d_pair(sa, &mapA, fb, kc, arow);
+            if constexpr (MODE == MODE_GATE_UP_CONCAT) {
+              // leader: the 128 gate columns; peer: the matching 128 up columns
+              const int c0 = tc.n * 128;
+              const int half = static_cast<int>(rank);
+              tma_load_4d_pair(sb, &mapB, fb, c0, half, kc, tc.e);
+              tma_load_4d_pair(sb + B_BOX_BYTES, &mapB, fb, c0 + 64, half, kc, tc.e);
+            } else {
+              const int c0 = tc.n * BN + static_cast<int>(rank) * 128;
+              tma_load_3d_pair(sb, &mapB, fb, c0, kc, tc.e);
+              tma_load_3d_pair(sb + B_BOX_BYTES, &mapB, fb, c0 + 64, kc, tc.e);
+            }
           }
           ++it;
         }
       }
       if (ok) {
-        // Tail: wait until the MMA warp has released every stage, so that no
+        // Tail: wait until the MMAs have released every stage, so that no
         // tcgen05.commit arrival lands after this CTA exits.
-        for (int i = 0; i < STAGES; ++i, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = static_cast<uint32_t>(it / STAGES) & 1u;
+        for (int i = 0; i < G::STAGES; ++i, ++it) {
+          const int s = it % G::STAGES;
+          const uint32_t ph = static_cast<uint32_t>(it / G::STAGES) & 1u;
           if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kTimeoutNs)) break;
         }
-      } else {
+      } else if (leader) {
         // Aborted: let the copies already issued land before shared memory
         // is released (time-bounded, independent of the abort flag).
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < G::STAGES; ++s) {
           if (it > s) {
-            const int last = s + ((it - 1 - s) / STAGES) * STAGES;
-            wait_time_only(full0 + 8 * s, static_cast<uint32_t>(last / STAGES) & 1u);
+            const int last = s + ((it - 1 - s) / G::STAGES) * G::STAGES;
+            wait_time_only(full0 + 8 * s, static_cast<uint32_t>(last / G::STAGES) & 1u);
           }
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // --------------------------------------------------- MMA issuer
       int it = 0, ti = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x, ++ti) {
+      for (int t = first_tile; ok && t < total_tiles; t += tile_stride, ++ti) {
         const int acc = ti & 1;
         const uint32_t aph = static_cast<uint32_t>(ti >> 1) & 1u;
         if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, abort_flag, kTimeoutNs)) {
@@ -381,14 +429,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < p.num_kb; ++kb) {
-          const int s = it % STAGES;
-          const uint32_t ph = static_cast<uint32_t>(it / STAGES) & 1u;
+          const int s = it % G::STAGES;
+          const uint32_t ph = static_cast<uint32_t>(it / G::STAGES) & 1u;
           if (!mbar_wait(full0 + 8 * s, ph, abort_flag, kTimeoutNs)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t sa = sbase + s * STAGE_BYTES;
+          const uint32_t sa = sbase + s * G::STAGE_BYTES;
           const uint32_t sb = sa + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
@@ -398,17 +446,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // B: N-major; 64-column blocks B_BOX_BYTES apart (LBO), 8-row K
             // groups 1024 B apart (SBO); a 16-row K step is 2048 B.
             const uint64_t b_desc = smem_desc_sw128(sb + kk * UMMA_K * 128, B_BOX_BYTES, 1024);
-            mma_bf16_ss(d_tmem, a_desc, b_desc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            if constexpr (PAIR == 2) mma_bf16_ss_pair(d_tmem, a_desc, b_desc, G::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            else mma_bf16_ss(d_tmem, a_desc, b_desc, G::IDESC, (kb | kk) != 0 ? 1u : 0u);
           }
-          mma_commit(empty0 + 8 * s);
+          if constexpr (PAIR == 2) mma_commit_pair(empty0 + 8 * s, 0x3);
+          else mma_commit(empty0 + 8 * s);
           ++it;
         }
         if (!ok) break;
-        mma_commit(tfull0 + 8 * acc);
+        if constexpr (PAIR == 2) mma_commit_pair(tfull0 + 8 * acc, 0x3);
+        else mma_commit(tfull0 + 8 * acc);
       }
       if (!ok) {
         // Aborted: every MMA issued so far must finish before TMEM is freed.
-        mma_commit(drain_bar);
+        if constexpr (PAIR == 2) mma_commit_pair(drain_bar, 0x1);
+        else mma_commit(drain_bar);
         wait_time_only(drain_bar, 0);
       }
     }
@@ -417,8 +469,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quad = warp & 3;  // this warp may access TMEM lanes 32*quad..+31
     const int row = quad * 32 + lane;
     int ti = 0;
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++ti) {
-      const TileCoord tc = decode_tile(t, p.n_tiles, p.E, s_mt, s_off);
+    for (int t = first_tile; t < total_tiles; t += tile_stride, ++ti) {
+      TileCoord tc = decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
+      if constexpr (PAIR == 2) {
+        tc.row0 += static_cast<int>(rank) * BM;
+        tc.rows -= static_cast<int>(rank) * BM;  // may be <= 0: nothing of this half is stored
+      }
       const int acc = ti & 1;
       const uint32_t aph = static_cast<uint32_t>(ti >> 1) & 1u;
       const bool got = mbar_wait(tfull0 + 8 * acc, aph, abort_flag, kTimeoutNs);
@@ -429,15 +485,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       else if constexpr (MODE == MODE_GATE_UP_INTERLEAVED) epilogue_gate_up_interleaved(p, tc, tacc, row);
       else epilogue_down(p, tc, tacc, row);
       tc_fence_before_sync();
-      mbar_arrive(tempty0 + 8 * acc);
+      if constexpr (PAIR == 2) mbar_arrive_cluster(map_to_rank(tempty0 + 8 * acc, 0));
+      else mbar_arrive(tempty0 + 8 * acc);
     }
   }
 
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, p.err_bit);
+  if constexpr (PAIR == 2) {
+    tc_fence_before_sync();
+    cluster_sync();  // neither CTA leaves while the other may still signal it
+  }
   if (warp == 1) {
+    __syncwarp();
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if constexpr (PAIR == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -468,8 +531,77 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, int rank, const cuuint6
   return r == CUDA_SUCCESS;
 }
 
+template <int PAIR>
 constexpr size_t smem_bytes_for(int E) {
-  return 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + CTRL_BYTES + 2 * static_cast<size_t>(E + 1) * 4;
+  return 1024 + static_cast<size_t>(Geo<PAIR>::STAGES) * Geo<PAIR>::STAGE_BYTES + CTRL_BYTES +
+         2 * static_cast<size_t>(E + 1) * 4;
+}
+
+// Clusters of two that can be resident at once (cached per kernel).
+template <int MODE>
+int max_pair_clusters(size_t smem, int num_sms) {
+  static int cached = 0;
+  if (cached > 0) return cached;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<MODE, 2>, &cfg) != cudaSuccess || n <= 0)
+    n = num_sms / 2;
+  cached = n;
+  return n;
+}
+
+// The CTA-pair variant keeps the tensor pipe busier per clock (86-91% vs
+// 76-79% of cycles on the Mixtral-shaped GEMMs) but these GEMMs run at the
+// part's power limit, where it draws more power, runs at a lower clock and
+// ends no faster; the single-CTA kernel is therefore the default.
+// MOE_B200_CTA_PAIR=2 selects the pair variant (1 forces the default).
+int choose_pair(int /*R*/, int /*E*/) {
+  if (const char* env = std::getenv("MOE_B200_CTA_PAIR")) {
+    if (env[0] == '2') return 2;
+  }
+  return 1;
+}
+
+template <int MODE, int PAIR>
+cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmParams& p, int num_sms,
+                        cudaStream_t stream) {
+  const int64_t max_pieces = p.R / Geo<PAIR>::PIECE + std::min(p.E, p.R);
+  const int64_t max_tiles = max_pieces * p.n_tiles;
+  const size_t smem = smem_bytes_for<PAIR>(p.E);
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_bytes_for<PAIR>(kMaxExperts)));
+  if (err != cudaSuccess) return err;
+  if constexpr (PAIR == 1) {
+    const int grid = static_cast<int>(std::min<int64_t>(max_tiles, num_sms));
+    grouped_gemm_kernel<MODE, 1><<<grid, NUM_THREADS, smem, stream>>>(mapA, mapB, p);
+    return cudaGetLastError();
+  } else {
+    const int clusters =
+        static_cast<int>(std::min<int64_t>(max_tiles, max_pair_clusters<MODE>(smem_bytes_for<2>(kMaxExperts), num_sms)));
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 2>, mapA, mapB, p);
+  }
 }
 
 template <int MODE>
@@ -518,15 +650,8 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t stream) {
   p.alpha = a.alpha;
   p.limit = a.limit;
   p.err_bit = down ? MOE_DEVICE_ERR_TIMEOUT_GEMM2 : MOE_DEVICE_ERR_TIMEOUT_GEMM1;
-  const int64_t max_pieces = a.R / BM + std::min(a.E, a.R);
-  const int64_t max_tiles = max_pieces * p.n_tiles;
-  const int grid = static_cast<int>(std::min<int64_t>(max_tiles, a.num_sms));
-  const size_t smem = smem_bytes_for(a.E);
-  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem_bytes_for(kMaxExperts)));
-  if (err != cudaSuccess) return err;
-  grouped_gemm_kernel<MODE><<<grid, NUM_THREADS, smem, stream>>>(mapA, mapB, p);
-  return cudaGetLastError();
+  if (choose_pair(a.R, a.E) == 2) return launch_with<MODE, 2>(mapA, mapB, p, a.num_sms, stream);
+  return launch_with<MODE, 1>(mapA, mapB, p, a.num_sms, stream);
 }
 
 }  // namespace

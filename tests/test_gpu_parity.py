@@ -35,6 +35,23 @@ def test_forward_small(name):
     run_and_check(SMALL[name], seed=0)
 
 
+@pytest.mark.parametrize("pair", ["1", "2"])
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_forward_small_each_cta_variant(name, pair, monkeypatch):
+    """Both GEMM variants on every layout: one CTA per 128x256 tile, or a CTA
+    pair on a 256x256 tile (tcgen05 cta_group::2)."""
+    monkeypatch.setenv("MOE_B200_CTA_PAIR", pair)
+    run_and_check(SMALL[name], seed=1)
+
+
+@pytest.mark.parametrize("pair", ["1", "2"])
+def test_forward_mixtral_shape_each_cta_variant(pair, monkeypatch):
+    monkeypatch.setenv("MOE_B200_CTA_PAIR", pair)
+    wl = WORKLOADS["mixtral"].replace(num_tokens=1024, hidden_dim=1024, moe_dim=1536,
+                                      logits_std=0.02 * math.sqrt(1024))
+    run_and_check(wl, seed=2)
+
+
 @pytest.mark.parametrize("seed", [1, 2])
 def test_forward_tiny_seeds(seed):
     run_and_check(WORKLOADS["tiny"], seed=seed)
