@@ -53,7 +53,7 @@ constexpr int A_BYTES = BM * BK * 2;            // 16 KB
 constexpr int B_BOX_BYTES = BK * 64 * 2;        // 8 KB: 64 K rows x 64 N columns
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;             // two BN-column fp32 accumulators
-constexpr int CTRL_BYTES = 256;
+constexpr int CTRL_BYTES = 512;  // mbarriers (bytes 0..255) and flags (256..)
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 
 // Per-CTA pipeline geometry.  PAIR = 1: one CTA computes a 128 x 256 tile and
@@ -260,9 +260,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tfull0 = empty0 + 8 * G::STAGES;     // 2 mbarriers
   const uint32_t tempty0 = tfull0 + 16;               // 2 mbarriers
   const uint32_t drain_bar = tempty0 + 16;            // 1 mbarrier
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 128);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 132);
-  int* bad_flag = reinterpret_cast<int*>(ctrl + 136);
+  static_assert((2 * G::STAGES + 5) * 8 <= 256, "mbarriers overflow their part of the control block");
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 256);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 260);
+  int* bad_flag = reinterpret_cast<int*>(ctrl + 264);
   int* s_off = reinterpret_cast<int*>(ctrl + CTRL_BYTES);
   int* s_mt = s_off + (p.E + 1);
 
