@@ -179,8 +179,10 @@ moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x, const void*
  * the routing kept in the workspace.  expert_indices_out [T,k],
  * expert_weights_out [T,k] and sink_weights_out [T,S] are optional copies of
  * the routing (NULL = not returned; sink_weights_out is written only when
- * S > 0).  Eight kernel launches, no host synchronisation, no allocation, so
- * the call can be captured in a CUDA graph. */
+ * S > 0).  Eight kernel launches (five when T*k <= 2048 and E <= 512: the
+ * router and the CSR build then share one single-CTA kernel), no host
+ * synchronisation, no allocation, so the call can be captured in a CUDA
+ * graph. */
 moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* logits,
                          const float* expert_bias, const float* global_scale, const void* gate_up_w,
                          const void* gate_up_b, const void* down_w, const void* down_b, void* out,

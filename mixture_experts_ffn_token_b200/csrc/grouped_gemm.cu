@@ -10,7 +10,7 @@
 //             down bias weighted with it as in NeMo _apply_bias), stored at
 //             the slot row so the k-way combine reads tokens in order.
 //
-// Kernel design (one persistent CTA per SM, 192 threads):
+// Kernel design (one persistent CTA per SM, 320 threads):
 //   warp 0      TMA producer: for every tile and 64-wide K block, one 128x64
 //               box of A (K-major, 128-byte swizzle) and four 64x64 boxes of
 //               B (N-major, 128-byte swizzle) into a 4-stage ring, completion
@@ -19,9 +19,10 @@
 //               tcgen05.mma 128x256x16 per stage (bf16 in, fp32 accumulate in
 //               TMEM) and tcgen05.commit's the stage back to the producer;
 //               two 256-column accumulators alternate between tiles;
-//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes (one output row
-//               per thread), bias + activation (gate_up) or bias x weight
-//               (down) in fp32, bf16 stores.
+//   warps 2..9  epilogue: tcgen05.ld of their 32 TMEM lanes (one output row
+//               per thread; two warps per lane quadrant split the columns),
+//               bias + activation (gate_up) or bias x weight (down) in fp32,
+//               bf16 stores.
 // Tiles are the ragged expert segments cut in 128-row pieces times the
 // output columns; the per-expert piece counts are rebuilt from the CSR
 // offsets in shared memory at kernel start, and CTAs walk the tile list with
@@ -51,7 +52,8 @@ constexpr int BK = 64;                  // K per stage: one 128-byte swizzle row
 constexpr int UMMA_K = 16;              // K per tcgen05.mma (kind::f16)
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB
 constexpr int B_BOX_BYTES = BK * 64 * 2;        // 8 KB: 64 K rows x 64 N columns
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_EPI_WARPS = 8;              // two per TMEM lane quadrant, each half the columns
+constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;  // producer warp, MMA warp, epilogue warps
 constexpr uint32_t TMEM_COLS = 512;             // two BN-column fp32 accumulators
 constexpr int CTRL_BYTES = 512;  // mbarriers (bytes 0..255) and flags (256..)
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
@@ -120,126 +122,139 @@ __device__ __forceinline__ bool wait_time_only(uint32_t bar, uint32_t parity) {
 }
 
 // ----------------------------------------------------------- epilogues
-// gate_up, concatenated [gate | up]: accumulator columns 0..127 are gate
-// columns hcol0.., columns 128..255 the matching up columns.
-__device__ __forceinline__ void epilogue_gate_up_concat(const GemmParams& p, const TileCoord& tc, uint32_t tacc,
-                                                        int row) {
-  const bool valid = row < tc.rows;
-  const int hcol0 = tc.n * 128;
-  const int64_t prow = static_cast<int64_t>(tc.row0) + row;
+// Each epilogue warp owns 32 tile rows (its TMEM lane quadrant) and half of
+// the tile's output columns, which it walks in chunks of 32 output columns:
+// every thread computes its row's 32 values from the fp32 accumulator, the
+// warp transposes them through a 32 x 32 bf16 staging block in shared
+// memory (row stride 80 B: conflict-free), then stores 8 rows x 64 B per
+// instruction, so each store fills whole 32-byte sectors of contiguous
+// columns instead of scattering 16-byte pieces over 32 rows.
+constexpr int kStageRowBytes = 80;
+constexpr int kStageWarpBytes = 32 * kStageRowBytes;  // 2560 B per epilogue warp
+constexpr int kOutChunk = 32;                          // output columns per chunk
+
+// gate_up: 32 h columns starting at tile h column hc (relative to the tile).
+template <int MODE>
+__device__ __forceinline__ void gate_up_chunk(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int hc,
+                                              uint32_t (&packed)[16]) {
+  const int hcol0 = tc.n * 128 + hc;  // absolute h column of value 0
   const __nv_bfloat16* bg = p.bias != nullptr ? p.bias + static_cast<int64_t>(tc.e) * 2 * p.D : nullptr;
-#pragma unroll 1
-  for (int c = 0; c < 128; c += 16) {
-    uint32_t g[16], u[16];
-    tmem_ld16(tacc + c, g);
-    tmem_ld16(tacc + 128 + c, u);
-    tmem_ld_wait();
+  uint32_t a0[32], a1[32];
+  if constexpr (MODE == MODE_GATE_UP_CONCAT) {
+    tmem_ld32(tacc + hc, a0);         // gate columns
+    tmem_ld32(tacc + 128 + hc, a1);   // matching up columns
+  } else {
+    tmem_ld32(tacc + 2 * hc, a0);     // (gate, up) pairs of h columns hc .. hc+15
+    tmem_ld32(tacc + 2 * hc + 32, a1);  // ... and hc+16 .. hc+31
+  }
+  tmem_ld_wait();
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int col = hcol0 + c + 8 * half;
-      if (valid && col < p.D) {
-        float hv[8];
+  for (int j = 0; j < 32; j += 2) {
+    float h2[2];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float gv = __uint_as_float(g[8 * half + j]);
-          float uv = __uint_as_float(u[8 * half + j]);
-          if (bg != nullptr) {
-            gv += __bfloat162float(bg[col + j]);
-            uv += __bfloat162float(bg[p.D + col + j]);
-          }
-          hv[j] = gated_act(p.activation, gv, uv, p.alpha, p.limit);
-        }
-        uint4 o;
-        o.x = pack_bf16x2(hv[0], hv[1]);
-        o.y = pack_bf16x2(hv[2], hv[3]);
-        o.z = pack_bf16x2(hv[4], hv[5]);
-        o.w = pack_bf16x2(hv[6], hv[7]);
-        *reinterpret_cast<uint4*>(p.out + prow * p.D + col) = o;
+    for (int q = 0; q < 2; ++q) {
+      const int jj = j + q;
+      float g, u;
+      if constexpr (MODE == MODE_GATE_UP_CONCAT) {
+        g = __uint_as_float(a0[jj]);
+        u = __uint_as_float(a1[jj]);
+      } else {
+        const uint32_t* src = jj < 16 ? a0 : a1;
+        const int m = jj & 15;
+        g = __uint_as_float(src[2 * m]);
+        u = __uint_as_float(src[2 * m + 1]);
       }
+      const int col = hcol0 + jj;
+      if (bg != nullptr && col < p.D) {
+        if constexpr (MODE == MODE_GATE_UP_CONCAT) {
+          g += __bfloat162float(bg[col]);
+          u += __bfloat162float(bg[p.D + col]);
+        } else {
+          g += __bfloat162float(bg[2 * col]);
+          u += __bfloat162float(bg[2 * col + 1]);
+        }
+      }
+      h2[q] = gated_act(p.activation, g, u, p.alpha, p.limit);
     }
+    packed[j / 2] = pack_bf16x2(h2[0], h2[1]);
   }
 }
 
-// gate_up, interleaved: accumulator columns (2j, 2j+1) are (gate, up) of h
-// column hcol0 + j.
-__device__ __forceinline__ void epilogue_gate_up_interleaved(const GemmParams& p, const TileCoord& tc, uint32_t tacc,
-                                                             int row) {
-  const bool valid = row < tc.rows;
-  const int hcol0 = tc.n * 128;
-  const int64_t prow = static_cast<int64_t>(tc.row0) + row;
-  const __nv_bfloat16* bg = p.bias != nullptr ? p.bias + static_cast<int64_t>(tc.e) * 2 * p.D : nullptr;
-#pragma unroll 1
-  for (int c = 0; c < 256; c += 32) {
-    uint32_t v[32];
-    tmem_ld16(tacc + c, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-    tmem_ld16(tacc + c + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-    tmem_ld_wait();
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int col = hcol0 + c / 2 + 8 * half;
-      if (valid && col < p.D) {
-        float hv[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float gv = __uint_as_float(v[16 * half + 2 * j]);
-          float uv = __uint_as_float(v[16 * half + 2 * j + 1]);
-          if (bg != nullptr) {
-            gv += __bfloat162float(bg[2 * (col + j)]);
-            uv += __bfloat162float(bg[2 * (col + j) + 1]);
-          }
-          hv[j] = gated_act(p.activation, gv, uv, p.alpha, p.limit);
-        }
-        uint4 o;
-        o.x = pack_bf16x2(hv[0], hv[1]);
-        o.y = pack_bf16x2(hv[2], hv[3]);
-        o.z = pack_bf16x2(hv[4], hv[5]);
-        o.w = pack_bf16x2(hv[6], hv[7]);
-        *reinterpret_cast<uint4*>(p.out + prow * p.D + col) = o;
-      }
-    }
-  }
-}
-
-// down: (acc + b_d[e]) * w[slot], stored at the slot's row of Y.
-__device__ __forceinline__ void epilogue_down(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int row) {
-  bool ok = row < tc.rows;
-  int slot = 0;
-  float wgt = 0.f;
-  if (ok) {
-    slot = p.perm[tc.row0 + row];
-    if (slot < 0 || slot >= p.R) {
-      atomicOr(p.status, MOE_DEVICE_ERR_CSR);
-      ok = false;
-    } else {
-      wgt = p.weights[slot];
-    }
-  }
-  const int col0 = tc.n * BN;
+// down: 32 output columns starting at tile column oc: (acc + b_d[e]) * w.
+__device__ __forceinline__ void down_chunk(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int oc,
+                                           float wgt, uint32_t (&packed)[16]) {
+  const int col0 = tc.n * BN + oc;
   const __nv_bfloat16* bd = p.bias != nullptr ? p.bias + static_cast<int64_t>(tc.e) * p.H : nullptr;
-  __nv_bfloat16* orow = p.out + static_cast<int64_t>(slot) * p.H;
+  uint32_t a[32];
+  tmem_ld32(tacc + oc, a);
+  tmem_ld_wait();
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    float y[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      float v = __uint_as_float(a[j + q]);
+      if (bd != nullptr && col0 + j + q < p.H) v += __bfloat162float(bd[col0 + j + q]);
+      y[q] = v * wgt;
+    }
+    packed[j / 2] = pack_bf16x2(y[0], y[1]);
+  }
+}
+
+// One tile's epilogue for one warp: rows quad*32.., output columns of `part`.
+template <int MODE>
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int quad,
+                                              int part, int lane, uint8_t* stage) {
+  constexpr bool kDown = MODE == MODE_DOWN;
+  const int row = quad * 32 + lane;
+  // destination row of this thread's tile row, or -1 if it is not stored
+  int64_t dst = -1;
+  float wgt = 0.f;
+  if (row < tc.rows) {
+    if constexpr (kDown) {
+      const int slot = p.perm[tc.row0 + row];
+      if (slot < 0 || slot >= p.R) {
+        atomicOr(p.status, MOE_DEVICE_ERR_CSR);
+      } else {
+        dst = static_cast<int64_t>(slot) * p.H;
+        wgt = p.weights[slot];
+      }
+    } else {
+      dst = (static_cast<int64_t>(tc.row0) + row) * p.D;
+    }
+  }
+  // the 4 rows this lane stores in the transposed phase: 8*i + lane/4
+  int64_t my_dst[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int src_lane = 8 * i + (lane >> 2);
+    const int lo = __shfl_sync(0xffffffffu, static_cast<int>(dst & 0xffffffff), src_lane);
+    const int hi = __shfl_sync(0xffffffffu, static_cast<int>(dst >> 32), src_lane);
+    my_dst[i] = (static_cast<int64_t>(hi) << 32) | static_cast<uint32_t>(lo);
+  }
+  const int limit = kDown ? p.H : p.D;
+  const int part_cols = kDown ? BN / 2 : 64;  // output columns per part
+  const int base_col = (kDown ? tc.n * BN : tc.n * 128) + part * part_cols;
+  const int q = lane & 3;  // 16-byte chunk of a 64-byte row segment
+  uint8_t* my_row = stage + lane * kStageRowBytes;
 #pragma unroll 1
-  for (int c = 0; c < BN; c += 32) {
-    uint32_t v[32];
-    tmem_ld16(tacc + c, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-    tmem_ld16(tacc + c + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-    tmem_ld_wait();
+  for (int oc = 0; oc < part_cols; oc += kOutChunk) {
+    uint32_t packed[16];
+    __syncwarp();
+    if constexpr (kDown) down_chunk(p, tc, tacc, part * part_cols + oc, wgt, packed);
+    else gate_up_chunk<MODE>(p, tc, tacc, part * part_cols + oc, packed);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int col = col0 + c + 8 * q;
-      if (ok && col < p.H) {
-        float y[8];
+    for (int c = 0; c < 4; ++c)
+      *reinterpret_cast<uint4*>(my_row + 16 * c) =
+          make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+    __syncwarp();
+    const int col = base_col + oc + 8 * q;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float a = __uint_as_float(v[8 * q + j]);
-          if (bd != nullptr) a += __bfloat162float(bd[col + j]);
-          y[j] = a * wgt;
-        }
-        uint4 o;
-        o.x = pack_bf16x2(y[0], y[1]);
-        o.y = pack_bf16x2(y[2], y[3]);
-        o.z = pack_bf16x2(y[4], y[5]);
-        o.w = pack_bf16x2(y[6], y[7]);
-        *reinterpret_cast<uint4*>(orow + col) = o;
+    for (int i = 0; i < 4; ++i) {
+      const int rr = 8 * i + (lane >> 2);
+      if (my_dst[i] >= 0 && col < limit) {
+        const uint4 v = *reinterpret_cast<const uint4*>(stage + rr * kStageRowBytes + 16 * q);
+        *reinterpret_cast<uint4*>(p.out + my_dst[i] + col) = v;
       }
     }
   }
@@ -266,6 +281,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   int* bad_flag = reinterpret_cast<int*>(ctrl + 264);
   int* s_off = reinterpret_cast<int*>(ctrl + CTRL_BYTES);
   int* s_mt = s_off + (p.E + 1);
+  // epilogue staging: one kStageWarpBytes block per epilogue warp, 16-byte aligned
+  uint8_t* s_stage = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(s_mt + p.E + 1) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -279,7 +297,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, 128 * PAIR);
+      mbar_init(tempty0 + 8 * a, 32 * NUM_EPI_WARPS * PAIR);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -468,7 +486,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ------------------------------------------------------ epilogue
     const int quad = warp & 3;  // this warp may access TMEM lanes 32*quad..+31
-    const int row = quad * 32 + lane;
+    const int part = (warp - 2) >> 2;  // which half of the tile's columns
     int ti = 0;
     for (int t = first_tile; t < total_tiles; t += tile_stride, ++ti) {
       TileCoord tc = decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
@@ -482,9 +500,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after_sync();
       const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
-      if constexpr (MODE == MODE_GATE_UP_CONCAT) epilogue_gate_up_concat(p, tc, tacc, row);
-      else if constexpr (MODE == MODE_GATE_UP_INTERLEAVED) epilogue_gate_up_interleaved(p, tc, tacc, row);
-      else epilogue_down(p, tc, tacc, row);
+      epilogue_tile<MODE>(p, tc, tacc, quad, part, lane, s_stage + (warp - 2) * kStageWarpBytes);
       tc_fence_before_sync();
       if constexpr (PAIR == 2) mbar_arrive_cluster(map_to_rank(tempty0 + 8 * acc, 0));
       else mbar_arrive(tempty0 + 8 * acc);
@@ -535,7 +551,7 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, int rank, const cuuint6
 template <int PAIR>
 constexpr size_t smem_bytes_for(int E) {
   return 1024 + static_cast<size_t>(Geo<PAIR>::STAGES) * Geo<PAIR>::STAGE_BYTES + CTRL_BYTES +
-         2 * static_cast<size_t>(E + 1) * 4;
+         2 * static_cast<size_t>(E + 1) * 4 + 16 + NUM_EPI_WARPS * kStageWarpBytes;
 }
 
 // Clusters of two that can be resident at once (cached per kernel).

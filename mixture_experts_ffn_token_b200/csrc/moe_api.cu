@@ -256,12 +256,25 @@ moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const void* lo
   float* w = w_out != nullptr ? w_out : at<float>(ws, L.w);
   float* sink = (sink_out != nullptr || cfg->num_sink == 0) ? sink_out : at<float>(ws, L.sink);
   if (ev != nullptr) cudaEventRecord(ev[0], stream);
-  const moe::RouterArgs ra = router_args(cfg, logits, expert_bias, global_scale, idx, w, sink, at<int>(ws, L.status));
-  if (moe::launch_router(ra, stream) != cudaSuccess) return MOE_ERR_CUDA;
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* perm = at<int32_t>(ws, L.perm);
-  if ((st = enqueue_csr(cfg, idx, offsets, perm, nullptr, ws, L, stream, ev != nullptr ? ev + 1 : nullptr)) != MOE_OK)
-    return st;
+  const int64_t R = static_cast<int64_t>(cfg->num_tokens) * cfg->top_k;
+  if (R <= moe::kSmallSlots && cfg->num_experts <= moe::kSmallExperts) {
+    // small (decode-sized) problems: routing and the CSR build in one CTA;
+    // the CSR stages then record back-to-back events
+    const moe::RouterArgs ra = router_args(cfg, logits, expert_bias, global_scale, idx, w, sink, nullptr);
+    if (moe::launch_route_csr_small(ra, offsets, perm, at<int>(ws, L.status), stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (ev != nullptr)
+      for (int i = 1; i <= 3; ++i) cudaEventRecord(ev[i], stream);
+  } else {
+    const moe::RouterArgs ra =
+        router_args(cfg, logits, expert_bias, global_scale, idx, w, sink, at<int>(ws, L.status));
+    if (moe::launch_router(ra, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((st = enqueue_csr(cfg, idx, offsets, perm, nullptr, ws, L, stream, ev != nullptr ? ev + 1 : nullptr)) !=
+        MOE_OK)
+      return st;
+  }
   return enqueue_ffn(cfg, x, gate_up_w, gate_up_b, down_w, down_b, offsets, perm, w, out, ws, L, num_sms, stream,
                      ev != nullptr ? ev + 4 : nullptr);
 }

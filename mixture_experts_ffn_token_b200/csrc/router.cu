@@ -39,14 +39,11 @@ __device__ __forceinline__ float load_logit(const void* logits, int64_t i) {
 
 __device__ __forceinline__ double log_sigmoid(double z) { return fmin(z, 0.0) - log1p(exp(-fabs(z))); }
 
+// Routes token t with the calling warp; returns this lane's selected expert
+// (lanes 0..k-1, in selection order) and writes idx, w and sink_w.
 template <int NPL, bool SINK, bool BF16>
-__global__ void __launch_bounds__(128) router_kernel(const RouterArgs a) {
-  if (a.status_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.status_reset = 0;
-  const int lane = threadIdx.x & 31;
-  const int t = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
-  if (t >= a.T) return;
+__device__ __forceinline__ int route_token(const RouterArgs& a, int t, int lane) {
   const int64_t row = static_cast<int64_t>(t) * a.stride;
-
   float key[NPL];
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
@@ -122,6 +119,104 @@ __global__ void __launch_bounds__(128) router_kernel(const RouterArgs a) {
   } else if (SINK && active) {
     a.sink_w[static_cast<int64_t>(t) * a.S + (lane - a.k)] = static_cast<float>(w);
   }
+  return my_e;
+}
+
+template <int NPL, bool SINK, bool BF16>
+__global__ void __launch_bounds__(128) router_kernel(const RouterArgs a) {
+  if (a.status_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.status_reset = 0;
+  const int lane = threadIdx.x & 31;
+  const int t = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
+  if (t >= a.T) return;
+  route_token<NPL, SINK, BF16>(a, t, lane);
+}
+
+// Small problems (R <= kSmallSlots, E <= kSmallExperts): routing and the
+// whole CSR build in one CTA of kSmallWarps warps, replacing four launches.
+// The CSR part is the counting sort of csr.cu with a single chunk: each warp
+// owns a run of consecutive slots, a per-warp histogram scanned across warps
+// and experts gives every slot its position, stable in slot order.
+template <int NPL, bool SINK, bool BF16>
+__global__ void __launch_bounds__(32 * kSmallWarps) route_csr_small_kernel(const RouterArgs a, int32_t* offsets,
+                                                                           int32_t* perm, int* status) {
+  extern __shared__ int sm[];
+  int* s_idx = sm;                           // [R]
+  int* wcnt = sm + kSmallSlots;              // [kSmallWarps][E]
+  __shared__ int warp_tot[kSmallWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int R = a.T * a.k, E = a.E;
+  if (threadIdx.x == 0) *status = 0;
+  for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) wcnt[i] = 0;
+  for (int t = warp; t < a.T; t += kSmallWarps) {
+    const int e = route_token<NPL, SINK, BF16>(a, t, lane);
+    if (lane < a.k) s_idx[t * a.k + lane] = e;
+  }
+  __syncthreads();
+  constexpr int kPerWarp = kSmallSlots / kSmallWarps;
+  const int wbase = warp * kPerWarp;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int* my = wcnt + warp * E;
+  bool bad = false;
+  for (int r = 0; r < kPerWarp; r += 32) {
+    const int s = wbase + r + lane;
+    const int e = s < R ? s_idx[s] : -1;
+    const bool ok = e >= 0 && e < E;
+    if (s < R && !ok) bad = true;
+    const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : E + lane);
+    if (ok && (peers & lt_mask) == 0) my[e] += __popc(peers);
+    __syncwarp();
+  }
+  if (bad) atomicOr(status, MOE_DEVICE_ERR_EXPERT_INDEX);
+  __syncthreads();
+  // per expert: exclusive prefix over warps, total, then exclusive scan over experts
+  const int e = threadIdx.x;  // blockDim.x == 32 * kSmallWarps >= E
+  int total = 0;
+  if (e < E) {
+    for (int w = 0; w < kSmallWarps; ++w) {
+      const int v = wcnt[w * E + e];
+      wcnt[w * E + e] = total;
+      total += v;
+    }
+  }
+  int incl = total;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = lane < kSmallWarps ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += y;
+    }
+    if (lane < kSmallWarps) warp_tot[lane] = v;
+  }
+  __syncthreads();
+  const int excl = incl - total + (warp > 0 ? warp_tot[warp - 1] : 0);
+  if (e < E) {
+    offsets[e] = excl;
+    for (int w = 0; w < kSmallWarps; ++w) wcnt[w * E + e] += excl;
+  }
+  if (e == E - 1) offsets[E] = excl + total;
+  __syncthreads();
+  for (int r = 0; r < kPerWarp; r += 32) {
+    const int s = wbase + r + lane;
+    const int ee = s < R ? s_idx[s] : -1;
+    const bool ok = ee >= 0 && ee < E;
+    const uint32_t peers = __match_any_sync(0xffffffffu, ok ? ee : E + lane);
+    int base = 0;
+    if (ok) base = my[ee];
+    __syncwarp();
+    if (ok) {
+      perm[base + __popc(peers & lt_mask)] = s;
+      if ((peers & lt_mask) == 0) my[ee] += __popc(peers);
+    }
+    __syncwarp();
+  }
 }
 
 template <int NPL>
@@ -139,7 +234,32 @@ cudaError_t launch_npl(const RouterArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+template <int NPL>
+cudaError_t launch_small_npl(const RouterArgs& a, int32_t* offsets, int32_t* perm, int* status,
+                             cudaStream_t stream) {
+  const size_t smem = (kSmallSlots + static_cast<size_t>(kSmallWarps) * a.E) * sizeof(int);
+  const dim3 block(32 * kSmallWarps);
+  if (a.sink) {
+    if (a.logits_bf16) route_csr_small_kernel<NPL, true, true><<<1, block, smem, stream>>>(a, offsets, perm, status);
+    else route_csr_small_kernel<NPL, true, false><<<1, block, smem, stream>>>(a, offsets, perm, status);
+  } else {
+    if (a.logits_bf16) route_csr_small_kernel<NPL, false, true><<<1, block, smem, stream>>>(a, offsets, perm, status);
+    else route_csr_small_kernel<NPL, false, false><<<1, block, smem, stream>>>(a, offsets, perm, status);
+  }
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_route_csr_small(const RouterArgs& a, int32_t* offsets, int32_t* perm, int* status,
+                                   cudaStream_t stream) {
+  const int per_lane = (a.E + 31) / 32;
+  if (per_lane <= 1) return launch_small_npl<1>(a, offsets, perm, status, stream);
+  if (per_lane <= 2) return launch_small_npl<2>(a, offsets, perm, status, stream);
+  if (per_lane <= 4) return launch_small_npl<4>(a, offsets, perm, status, stream);
+  if (per_lane <= 8) return launch_small_npl<8>(a, offsets, perm, status, stream);
+  return launch_small_npl<16>(a, offsets, perm, status, stream);
+}
 
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t stream) {
   if (a.T <= 0) return cudaSuccess;

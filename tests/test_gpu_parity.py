@@ -64,6 +64,8 @@ def test_forward_tiny_seeds(seed):
     dict(activation="silu", limit=0.05),                        # clamps active on N(0,.) projections
     dict(activation="swigluoai", alpha=1.702, limit=0.05, has_bias=True),
     dict(num_tokens=200, hidden_dim=8, moe_dim=8),              # single partial K block, tiny N
+    dict(num_tokens=1100),                                      # R > 2048: separate router and CSR kernels
+    dict(num_experts=600, num_tokens=40, logits_std=1.0),       # E > 512: separate router and CSR kernels
 ])
 def test_forward_edge_cases(variant):
     run_and_check(WORKLOADS["tiny"].replace(**variant), seed=3)
