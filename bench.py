@@ -57,10 +57,11 @@ def max_over_ranks(x, dist_mod, device):
 
 
 def launches_per_step(wl):
-    """Kernels one moe_forward launches: the router and the 3-kernel CSR build
-    share one kernel when T*k <= 2048 and E <= 512."""
+    """Kernels one call launches: router + 3-kernel CSR build (one kernel
+    when T*k <= 2048 and E <= 512), gather, two grouped GEMMs, combine, and
+    with shared experts their index, gather and two GEMMs."""
     small = wl.num_tokens * wl.top_k <= 2048 and wl.num_experts <= 512
-    return 5 if small else 8
+    return (1 if small else 4) + 3 + (4 if wl.num_shared > 0 else 0) + 1
 
 
 def job_throughput(world, tokens_per_rank, ms_per_step):
@@ -88,7 +89,8 @@ def workload_bytes(wl):
 
 def touched_expert_bytes(wl, idx):
     used = torch.unique(idx.reshape(-1)).numel()
-    return used * 3 * wl.hidden_dim * wl.moe_dim * 2, used
+    shared = wl.num_shared * 3 * wl.hidden_dim * wl.shared_dim * 2
+    return used * 3 * wl.hidden_dim * wl.moe_dim * 2 + shared, used
 
 
 class ClockSampler:
@@ -192,15 +194,24 @@ def oracle_sample_rate(wl, inp_host, n_tokens, seed=0):
         idx, w = oracle.route_softmax_topk(logits, wl.num_experts, wl.top_k)
     else:
         bias = None if inp_host["expert_bias"] is None else inp_host["expert_bias"].numpy()
-        idx, w, _ = oracle.route_sigmoid_sink(logits, wl.num_experts, wl.num_sink, wl.top_k, bias,
-                                              wl.route_scale, float(inp_host["global_scale"][0]))
+        idx, w, sw = oracle.route_sigmoid_sink(logits, wl.num_experts, wl.num_sink, wl.top_k, bias,
+                                               wl.route_scale, float(inp_host["global_scale"][0]))
     full_idx = np.zeros((wl.num_tokens, wl.top_k), np.int32)
     full_w = np.zeros((wl.num_tokens, wl.top_k))
     full_idx[toks] = idx
     full_w[toks] = w
+    mask = None if inp_host.get("token_mask") is None else inp_host["token_mask"].numpy()
     oracle.expert_ffn(inp_host["x_bits"], full_idx, full_w, inp_host["W_gu_bits"], inp_host["W_d_bits"],
                       inp_host["b_gu_bits"], inp_host["b_d_bits"], wl.gate_up_format, wl.activation, wl.alpha,
-                      wl.limit, tokens=toks)
+                      wl.limit, tokens=toks, weight_first=wl.weight_first, token_mask=mask)
+    if wl.num_shared > 0:
+        gates = np.ones((wl.num_tokens, wl.num_shared))
+        if wl.router == "sigmoid_sink":
+            gates[toks] = sw
+        oracle.shared_expert_ffn(inp_host["x_bits"], gates, bf16_bits(inp_host["Ws_gu"]), bf16_bits(inp_host["Ws_d"]),
+                                 bf16_bits(inp_host.get("bs_gu")), bf16_bits(inp_host.get("bs_d")),
+                                 wl.gate_up_format, wl.activation, wl.alpha, wl.limit, tokens=toks,
+                                 weight_first=wl.weight_first, token_mask=mask)
     dt = time.perf_counter() - t0
     return n_tokens / dt, dt, oracle.num_threads()
 
@@ -299,12 +310,18 @@ def timed_steps(step, steps, stream, flush):
     return total
 
 
-def run_e2e(args, cfg, inp, kw, ws, stream, dist):
-    """K steps of moe_forward fed from, and returning to, pinned host memory.
+def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None):
+    """K steps of moe_forward (moe_forward_ex when `make_ex` builds its extras
+    from a device token mask) fed from, and returning to, pinned host memory.
+    The token mask, when there is one, is a per-step input and is copied too.
     Returns the device time (max over ranks) of the whole region in ms."""
     T, H = inp["x"].shape
     x_h = inp["x"].cpu().pin_memory()
     lg_h = inp["logits"].cpu().pin_memory()
+    has_mask = inp["token_mask"] is not None
+    mask_h = inp["token_mask"].cpu().pin_memory() if has_mask else None
+    mask_d = [torch.empty_like(inp["token_mask"]) if has_mask else None for _ in range(2)]
+    ex_b = [make_ex(mask_d[b]) if make_ex is not None else None for b in range(2)]
     out_h = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     x_d = [torch.empty_like(inp["x"]) for _ in range(2)]
     lg_d = [torch.empty_like(inp["logits"]) for _ in range(2)]
@@ -326,11 +343,17 @@ def run_e2e(args, cfg, inp, kw, ws, stream, dist):
                     h2d.wait_event(fwd_done[i - 2])        # buffer b no longer read by step i-2
                 x_d[b].copy_(x_h, non_blocking=True)
                 lg_d[b].copy_(lg_h, non_blocking=True)
+                if has_mask:
+                    mask_d[b].copy_(mask_h, non_blocking=True)
                 in_ready[i].record(h2d)
             stream.wait_event(in_ready[i])
             if i >= 2:
                 stream.wait_event(out_done[i - 2])         # out_d[b] copied out by step i-2
-            abi.moe_forward(cfg, x_d[b], lg_d[b], inp["W_gu"], inp["W_d"], out_d[b], ws, stream=stream, **kw)
+            if ex_b[b] is None:
+                abi.moe_forward(cfg, x_d[b], lg_d[b], inp["W_gu"], inp["W_d"], out_d[b], ws, stream=stream, **kw)
+            else:
+                abi.moe_forward_ex(cfg, ex_b[b], x_d[b], lg_d[b], inp["W_gu"], inp["W_d"], out_d[b], ws,
+                                   stream=stream, **kw)
             fwd_done[i].record(stream)
             with torch.cuda.stream(d2h):
                 d2h.wait_event(fwd_done[i])
@@ -366,7 +389,17 @@ def run_gpu(args, wl):
     cfg = abi.make_config(wl)
     inp = make_inputs(wl, seed=rank, device="cuda")
     T, H, k, S, E = wl.num_tokens, wl.hidden_dim, wl.top_k, wl.num_sink, wl.num_experts
-    ws = torch.empty(abi.moe_workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    extras = make_ex = None
+    if wl.extended:
+        def make_ex(mask):
+            return abi.make_extras(token_mask=mask, apply_router_weight_first=wl.weight_first,
+                                   shared_gate_up_w=inp.get("Ws_gu"), shared_down_w=inp.get("Ws_d"),
+                                   shared_gate_up_b=inp.get("bs_gu"), shared_down_b=inp.get("bs_d"))
+        extras = make_ex(inp["token_mask"])
+        ws_bytes = abi.moe_workspace_size_ex(cfg, extras)
+    else:
+        ws_bytes = abi.moe_workspace_size(cfg)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
     out = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
     idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
     w = torch.empty((T, k), dtype=torch.float32, device="cuda")
@@ -378,7 +411,10 @@ def run_gpu(args, wl):
               global_scale=inp["global_scale"], expert_indices_out=idx, expert_weights_out=w, sink_weights_out=sink)
 
     def step(evs=None):
-        if evs is None:
+        if extras is not None:
+            abi.moe_forward_ex(cfg, extras, inp["x"], inp["logits"], inp["W_gu"], inp["W_d"], out, ws, events=evs,
+                               **kw)
+        elif evs is None:
             abi.moe_forward(cfg, inp["x"], inp["logits"], inp["W_gu"], inp["W_d"], out, ws, **kw)
         else:
             abi.moe_forward_timed(cfg, evs, inp["x"], inp["logits"], inp["W_gu"], inp["W_d"], out, ws, **kw)
@@ -408,7 +444,7 @@ def run_gpu(args, wl):
     # durations for the roofline come from here (a timing event between two
     # kernels stops them overlapping, so the step total above is taken
     # without them)
-    n_ev = abi.NUM_STAGE_EVENTS
+    n_ev = abi.NUM_STAGE_EVENTS_EX if extras is not None else abi.NUM_STAGE_EVENTS
     ev_sets = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     for evs in ev_sets:          # create the CUDA events outside the region
         for ev in evs:
@@ -428,17 +464,20 @@ def run_gpu(args, wl):
     # from pinned memory and its output device->host inside the timed region.
     # Copies run on their own streams, double-buffered, so step i's copies
     # overlap the compute of its neighbours.
-    e2e_ms = run_e2e(args, cfg, inp, kw, ws, stream, dist)
+    e2e_ms = run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex)
     e2e_value = job_throughput(world, T, e2e_ms / args.steps)
     x_h_bytes = inp["x"].numel() * 2 + inp["logits"].numel() * 4
+    if inp["token_mask"] is not None:
+        x_h_bytes += inp["token_mask"].numel()
     out_bytes = T * H * 2
 
     # ---------------- roofline of the dominant kernel
-    names = abi.STAGE_NAMES
+    names = abi.STAGE_NAMES_EX if extras is not None else abi.STAGE_NAMES
     flops = wl.flops()
     wbytes, used = touched_expert_bytes(wl, idx)
     gate_up_flops = 4 * T * k * H * wl.moe_dim
     down_flops = 2 * T * k * H * wl.moe_dim
+    shared_rows = T * wl.num_shared
     dom = max(range(len(names)), key=lambda i: stage_ms[i])
     dom_name = names[dom]
     clock_summary = clocks.summary()
@@ -447,9 +486,14 @@ def run_gpu(args, wl):
     capped = "sw_power_cap" in clock_summary.get("reasons", [])
     bf16_peak = peaks.get("bf16_tflops_sustained" if capped else "bf16_tflops", peaks.get("bf16_tflops"))
     bf16_kind = "sustained" if capped else "burst"
-    if dom_name in ("gemm_gate_up", "gemm_down"):
-        kflops = gate_up_flops if dom_name == "gemm_gate_up" else down_flops
-        kbytes = (2 if dom_name == "gemm_gate_up" else 1) * used * H * wl.moe_dim * 2
+    if dom_name in ("gemm_gate_up", "gemm_down", "shared_gemm_gate_up", "shared_gemm_down"):
+        up = dom_name.endswith("gate_up")
+        if dom_name.startswith("shared"):
+            kflops = (4 if up else 2) * shared_rows * H * wl.shared_dim
+            kbytes = (2 if up else 1) * wl.num_shared * H * wl.shared_dim * 2
+        else:
+            kflops = gate_up_flops if up else down_flops
+            kbytes = (2 if up else 1) * used * H * wl.moe_dim * 2
         t_flop = kflops / (bf16_peak * 1e12)
         t_byte = kbytes / (peaks["hbm_gbs"] * 1e9)
         if t_flop >= t_byte:

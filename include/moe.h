@@ -209,6 +209,59 @@ moe_status_t moe_forward_timed(const moe_config_t* cfg, const void* x, const voi
  * (other bits are reported through *device_status only). */
 moe_status_t moe_device_status(const void* workspace, int32_t* device_status, moe_stream_t stream);
 
+/* Extensions of the layer beyond the core path (moe_forward_ex).  A zeroed
+ * struct (or a NULL pointer) means none of them.
+ *   token_mask     [T] uint8 or NULL (NeMo GroupedExperts.forward token_mask):
+ *                  a token whose byte is 0 is still routed (its routing is
+ *                  returned) but goes through no expert and its output row
+ *                  is zero.
+ *   apply_router_weight_first  0 or 1 (StackedMoE apply_router_weight_first):
+ *                  1 scales each routed copy of x by its routing weight
+ *                  before the expert (rounded to bf16), so the expert's down
+ *                  bias is not weighted; 0 weights the expert's output.
+ *   num_shared, shared_dim, shared_*  (StackedMoE has_shared_experts,
+ *                  shared_experts_dim): num_shared dense experts that every
+ *                  token goes through, weights laid out like the routed ones:
+ *                  shared_gate_up_w [Ns, H, 2*Ds], shared_down_w [Ns, Ds, H],
+ *                  biases [Ns, 2*Ds] / [Ns, H] per has_bias (same gate/up
+ *                  format and activation as the routed experts).  With the
+ *                  sink router their gates are the sink weights (the sink
+ *                  lanes are gated shared experts, so num_shared must equal
+ *                  num_sink); with the softmax router their gate is 1.
+ *                  shared_dim must be a multiple of 8. */
+typedef struct {
+  const uint8_t* token_mask;
+  int32_t apply_router_weight_first;
+  int32_t num_shared;
+  int32_t shared_dim;
+  const void* shared_gate_up_w;
+  const void* shared_gate_up_b;
+  const void* shared_down_w;
+  const void* shared_down_b;
+} moe_extras_t;
+
+/* Events moe_forward_ex() records when given stage_events: router, CSR
+ * count, scan, scatter, gather, gate_up GEMM, down GEMM, shared index,
+ * shared gather, shared gate_up GEMM, shared down GEMM, combine, end.
+ * Stages that do not run record back to back. */
+#define MOE_NUM_STAGE_EVENTS_EX 13
+
+/* Workspace for moe_forward_ex with these extensions (adds, with shared
+ * experts, the [T*Ns] slot CSR, Xp_s/Y_s [T*Ns, H] and h_s [T*Ns, Ds]). */
+moe_status_t moe_workspace_size_ex(const moe_config_t* cfg, const moe_extras_t* extras, size_t* bytes);
+
+/* moe_forward with the extensions above.  Same arguments and conventions as
+ * moe_forward, plus `extras` (NULL = none) and stage_events (NULL, or
+ * MOE_NUM_STAGE_EVENTS_EX caller-created cudaEvent_t).  The output is
+ *   out[t] = mask[t] * ( sum_j  w_tj * FFN_e(tj)(x_t)          (or FFN(w_tj x_t))
+ *                      + sum_i  g_ti * SharedFFN_i(x_t) )      (or SharedFFN_i(g_ti x_t))
+ * summed in fp32 (routed slots j ascending, then shared i ascending). */
+moe_status_t moe_forward_ex(const moe_config_t* cfg, const moe_extras_t* extras, const void* x, const void* logits,
+                            const float* expert_bias, const float* global_scale, const void* gate_up_w,
+                            const void* gate_up_b, const void* down_w, const void* down_b, void* out,
+                            int32_t* expert_indices_out, float* expert_weights_out, float* sink_weights_out,
+                            void* workspace, size_t workspace_bytes, moe_stream_t stream, void* const* stage_events);
+
 /* moe_create_indices without a workspace.  This entry point has no
  * counterpart on the documentation pages; it exists for callers that cannot
  * allocate device memory at the point where they build the routing: code

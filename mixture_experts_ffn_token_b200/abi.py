@@ -31,7 +31,11 @@ NUM_STAGE_EVENTS = 9
 STAGE_NAMES = ("router", "csr_count", "csr_scan", "csr_scatter", "gather", "gemm_gate_up", "gemm_down", "combine")
 
 EXPORTED = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_create_indices", "moe_grouped_ffn",
-            "moe_forward", "moe_forward_timed", "moe_device_status", "moe_create_indices_noalloc")
+            "moe_forward", "moe_forward_timed", "moe_device_status", "moe_create_indices_noalloc",
+            "moe_workspace_size_ex", "moe_forward_ex")
+NUM_STAGE_EVENTS_EX = 13
+STAGE_NAMES_EX = ("router", "csr_count", "csr_scan", "csr_scatter", "gather", "gemm_gate_up", "gemm_down",
+                  "shared_index", "shared_gather", "shared_gemm_gate_up", "shared_gemm_down", "combine")
 
 
 class MoEConfig(ctypes.Structure):
@@ -53,6 +57,36 @@ class MoEConfig(ctypes.Structure):
         ("limit", ctypes.c_float),
         ("has_bias", ctypes.c_int32),
     ]
+
+
+class MoEExtras(ctypes.Structure):
+    """moe_extras_t."""
+    _fields_ = [
+        ("token_mask", ctypes.c_void_p),
+        ("apply_router_weight_first", ctypes.c_int32),
+        ("num_shared", ctypes.c_int32),
+        ("shared_dim", ctypes.c_int32),
+        ("shared_gate_up_w", ctypes.c_void_p),
+        ("shared_gate_up_b", ctypes.c_void_p),
+        ("shared_down_w", ctypes.c_void_p),
+        ("shared_down_b", ctypes.c_void_p),
+    ]
+
+
+def make_extras(token_mask=None, apply_router_weight_first=False, shared_gate_up_w=None, shared_down_w=None,
+                shared_gate_up_b=None, shared_down_b=None) -> MoEExtras:
+    """moe_extras_t from torch tensors (shared weights [Ns, H, 2Ds] / [Ns, Ds, H])."""
+    ex = MoEExtras()
+    ex.token_mask = None if token_mask is None else token_mask.data_ptr()
+    ex.apply_router_weight_first = 1 if apply_router_weight_first else 0
+    if shared_gate_up_w is not None:
+        ex.num_shared = shared_gate_up_w.shape[0]
+        ex.shared_dim = shared_gate_up_w.shape[2] // 2
+        ex.shared_gate_up_w = shared_gate_up_w.data_ptr()
+        ex.shared_down_w = shared_down_w.data_ptr()
+        ex.shared_gate_up_b = None if shared_gate_up_b is None else shared_gate_up_b.data_ptr()
+        ex.shared_down_b = None if shared_down_b is None else shared_down_b.data_ptr()
+    return ex
 
 
 class MoEError(RuntimeError):
@@ -91,6 +125,11 @@ def load_library():
     lib.moe_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
     lib.moe_create_indices_noalloc.restype = ctypes.c_int
     lib.moe_create_indices_noalloc.argtypes = [cfgp, vp, vp, vp, vp, vp]
+    exp = ctypes.POINTER(MoEExtras)
+    lib.moe_workspace_size_ex.restype = ctypes.c_int
+    lib.moe_workspace_size_ex.argtypes = [cfgp, exp, ctypes.POINTER(ctypes.c_size_t)]
+    lib.moe_forward_ex.restype = ctypes.c_int
+    lib.moe_forward_ex.argtypes = [cfgp, exp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
     _lib = lib
     return lib
 
@@ -195,6 +234,34 @@ def moe_forward_timed(cfg, events, x, logits, gate_up_w, down_w, out, workspace,
                                             _p(out), _p(expert_indices_out), _p(expert_weights_out),
                                             _p(sink_weights_out), _p(workspace), workspace.numel(),
                                             _stream(stream), arr), "moe_forward_timed")
+
+
+def moe_workspace_size_ex(cfg: MoEConfig, extras: Optional[MoEExtras]) -> int:
+    n = ctypes.c_size_t(0)
+    ex = None if extras is None else ctypes.byref(extras)
+    _check(load_library().moe_workspace_size_ex(ctypes.byref(cfg), ex, ctypes.byref(n)), "moe_workspace_size_ex")
+    return n.value
+
+
+def moe_forward_ex(cfg, extras, x, logits, gate_up_w, down_w, out, workspace, gate_up_b=None, down_b=None,
+                   expert_bias=None, global_scale=None, expert_indices_out=None, expert_weights_out=None,
+                   sink_weights_out=None, events=None, stream=None):
+    """moe_forward with token mask / router weight first / shared experts
+    (`extras`, a MoEExtras or None); `events`: None or 13 torch.cuda.Event."""
+    arr = None
+    if events is not None:
+        if len(events) != NUM_STAGE_EVENTS_EX:
+            raise ValueError(f"moe_forward_ex needs {NUM_STAGE_EVENTS_EX} events")
+        for ev in events:
+            if ev.cuda_event == 0:
+                ev.record(stream)
+        arr = (ctypes.c_void_p * NUM_STAGE_EVENTS_EX)(*[ev.cuda_event for ev in events])
+    ex = None if extras is None else ctypes.byref(extras)
+    _check(load_library().moe_forward_ex(ctypes.byref(cfg), ex, _p(x), _p(logits), _p(expert_bias),
+                                         _p(global_scale), _p(gate_up_w), _p(gate_up_b), _p(down_w), _p(down_b),
+                                         _p(out), _p(expert_indices_out), _p(expert_weights_out),
+                                         _p(sink_weights_out), _p(workspace), workspace.numel(), _stream(stream),
+                                         arr), "moe_forward_ex")
 
 
 def moe_device_status(workspace, stream=None) -> int:

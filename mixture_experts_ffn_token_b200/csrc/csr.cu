@@ -14,6 +14,8 @@
 //           32-slot step, a per-warp count table (scanned across warps) gives
 //           the position of each slot, so the order inside an expert is the
 //           slot order and no atomic decides any position.
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace moe {
@@ -23,8 +25,14 @@ constexpr int kCsrWarps = kCsrThreads / 32;
 constexpr int kSlotsPerWarp = kCsrChunk / kCsrWarps;  // 128
 static_assert(kSlotsPerWarp % 32 == 0, "slots per warp must be whole warp steps");
 
+// A slot takes part unless its token is masked out (mask may be null).
+__device__ __forceinline__ bool slot_live(const uint8_t* mask, int64_t s, int k) {
+  return mask == nullptr || mask[s / k] != 0;
+}
+
 __global__ void __launch_bounds__(kCsrThreads) csr_count_kernel(const int32_t* __restrict__ idx, int R, int E,
-                                                                int32_t* __restrict__ chunk_counts, int* status) {
+                                                                int32_t* __restrict__ chunk_counts, int* status,
+                                                                const uint8_t* __restrict__ mask, int k) {
   extern __shared__ int cnt[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
@@ -32,6 +40,7 @@ __global__ void __launch_bounds__(kCsrThreads) csr_count_kernel(const int32_t* _
   const int64_t end = min(base + kCsrChunk, static_cast<int64_t>(R));
   bool bad = false;
   for (int64_t s = base + threadIdx.x; s < end; s += blockDim.x) {
+    if (!slot_live(mask, s, k)) continue;
     const int e = idx[s];
     if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
     else bad = true;
@@ -87,7 +96,8 @@ __global__ void __launch_bounds__(1024) csr_scan_kernel(const int32_t* __restric
 __global__ void __launch_bounds__(kCsrThreads) csr_scatter_kernel(const int32_t* __restrict__ idx, int R, int E,
                                                                   const int32_t* __restrict__ chunk_base,
                                                                   int32_t* __restrict__ perm,
-                                                                  int32_t* __restrict__ inv) {
+                                                                  int32_t* __restrict__ inv,
+                                                                  const uint8_t* __restrict__ mask, int k) {
   extern __shared__ int wcnt[];  // [kCsrWarps][E]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kCsrWarps * E; i += blockDim.x) wcnt[i] = 0;
@@ -98,7 +108,7 @@ __global__ void __launch_bounds__(kCsrThreads) csr_scatter_kernel(const int32_t*
   // pass 1: per-warp histogram
   for (int r = 0; r < kSlotsPerWarp; r += 32) {
     const int64_t s = wbase + r + lane;
-    const int e = s < R ? idx[s] : -1;
+    const int e = s < R && slot_live(mask, s, k) ? idx[s] : -1;
     const bool ok = e >= 0 && e < E;
     const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : E + lane);
     if (ok && (peers & lt_mask) == 0) my[e] += __popc(peers);
@@ -119,7 +129,7 @@ __global__ void __launch_bounds__(kCsrThreads) csr_scatter_kernel(const int32_t*
   const int32_t* cb = chunk_base + static_cast<int64_t>(blockIdx.x) * E;
   for (int r = 0; r < kSlotsPerWarp; r += 32) {
     const int64_t s = wbase + r + lane;
-    const int e = s < R ? idx[s] : -1;
+    const int e = s < R && slot_live(mask, s, k) ? idx[s] : -1;
     const bool ok = e >= 0 && e < E;
     const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : E + lane);
     int base = 0;
@@ -135,11 +145,13 @@ __global__ void __launch_bounds__(kCsrThreads) csr_scatter_kernel(const int32_t*
   }
 }
 
-// One warp per gathered row: Xp[p, :] = x[perm[p] / k, :], 16-byte vectors.
+// One warp per gathered row: Xp[p, :] = x[perm[p] / k, :] (times
+// scale[perm[p]] when scale is given), 16-byte vectors.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ x,
                                                           const int32_t* __restrict__ perm,
                                                           const int32_t* __restrict__ offsets, int E, int R, int k,
-                                                          int H, __nv_bfloat16* __restrict__ Xp, int* status) {
+                                                          int H, const float* __restrict__ scale,
+                                                          __nv_bfloat16* __restrict__ Xp, int* status) {
   int total = offsets[E];
   if (total < 0 || total > R) {
     if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, MOE_DEVICE_ERR_CSR);
@@ -156,12 +168,30 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
     }
     const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(s / k) * H);
     uint4* dst = reinterpret_cast<uint4*>(Xp + p * H);
-    for (int c = lane; c < vec; c += 32) dst[c] = __ldg(src + c);
+    if (scale == nullptr) {
+      for (int c = lane; c < vec; c += 32) dst[c] = __ldg(src + c);
+    } else {
+      // apply_router_weight_first: the routing weight scales the expert input
+      const float f = scale[s];
+      for (int c = lane; c < vec; c += 32) {
+        const uint4 v = __ldg(src + c);
+        uint4 o;
+        o.x = pack_bf16x2(bf16_lo(v.x) * f, bf16_hi(v.x) * f);
+        o.y = pack_bf16x2(bf16_lo(v.y) * f, bf16_hi(v.y) * f);
+        o.z = pack_bf16x2(bf16_lo(v.z) * f, bf16_hi(v.z) * f);
+        o.w = pack_bf16x2(bf16_lo(v.w) * f, bf16_hi(v.w) * f);
+        dst[c] = o;
+      }
+    }
   }
 }
 
-// out[t, :] = sum_j Y[t*k + j, :] in fp32, j ascending, rounded to bf16.
+// out[t, :] = sum_j Y[t*k + j, :] (+ sum_i Ys[t*Ns + i, :] for shared
+// experts) in fp32, j then i ascending, rounded to bf16; a masked token's row
+// is zero.
 __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ Y, int T, int H, int k,
+                                                      const __nv_bfloat16* __restrict__ Ys, int Ns,
+                                                      const uint8_t* __restrict__ mask,
                                                       __nv_bfloat16* __restrict__ out) {
   const int vec = H / 8;
   const int64_t n = static_cast<int64_t>(T) * vec;
@@ -170,13 +200,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
     const int64_t t = i / vec;
     const int c = static_cast<int>(i - t * vec);
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < k; ++j) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(Y + (t * k + j) * H) + c);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    if (mask == nullptr || mask[t] != 0) {
+      for (int j = 0; j < k + Ns; ++j) {
+        const __nv_bfloat16* row = j < k ? Y + (t * k + j) * H : Ys + (t * Ns + (j - k)) * H;
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(row) + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        acc[2 * q] += bf16_lo(w[q]);
-        acc[2 * q + 1] += bf16_hi(w[q]);
+        for (int q = 0; q < 4; ++q) {
+          acc[2 * q] += bf16_lo(w[q]);
+          acc[2 * q + 1] += bf16_hi(w[q]);
+        }
       }
     }
     uint4 o;
@@ -188,13 +221,34 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
   }
 }
 
+// Shared experts as a grouped problem: expert i's segment is every token in
+// order, offsets[i] = i*T, and row i*T + t is slot t*Ns + i of the [T, Ns]
+// slot space (so slot / Ns is the token and the gates are indexed by slot).
+__global__ void __launch_bounds__(256) shared_index_kernel(int T, int Ns, int32_t* __restrict__ offsets,
+                                                           int32_t* __restrict__ perm) {
+  const int64_t n = static_cast<int64_t>(T) * Ns;
+  for (int64_t p = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; p < n;
+       p += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t i = p / T, t = p - i * T;
+    perm[p] = static_cast<int32_t>(t * Ns + i);
+  }
+  if (blockIdx.x == 0 && threadIdx.x <= Ns) offsets[threadIdx.x] = threadIdx.x * T;
+}
+
 }  // namespace
 
+cudaError_t launch_shared_index(int T, int Ns, int32_t* offsets, int32_t* perm, int num_sms, cudaStream_t stream) {
+  const int64_t n = static_cast<int64_t>(T) * Ns;
+  const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, num_sms * 4)));
+  shared_index_kernel<<<blocks, 256, 0, stream>>>(T, Ns, offsets, perm);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_csr_count(const int32_t* idx, int R, int E, int32_t* chunk_counts, int* status,
-                             cudaStream_t stream) {
+                             const uint8_t* mask, int k, cudaStream_t stream) {
   const int nchunks = csr_num_chunks(R);
   if (nchunks == 0) return cudaSuccess;
-  csr_count_kernel<<<nchunks, kCsrThreads, E * sizeof(int), stream>>>(idx, R, E, chunk_counts, status);
+  csr_count_kernel<<<nchunks, kCsrThreads, E * sizeof(int), stream>>>(idx, R, E, chunk_counts, status, mask, k);
   return cudaGetLastError();
 }
 
@@ -205,7 +259,7 @@ cudaError_t launch_csr_scan(const int32_t* chunk_counts, int nchunks, int E, int
 }
 
 cudaError_t launch_csr_scatter(const int32_t* idx, int R, int E, const int32_t* chunk_base, int32_t* perm,
-                               int32_t* inv, cudaStream_t stream) {
+                               int32_t* inv, const uint8_t* mask, int k, cudaStream_t stream) {
   const int nchunks = csr_num_chunks(R);
   if (nchunks == 0) return cudaSuccess;
   const size_t smem = static_cast<size_t>(kCsrWarps) * E * sizeof(int);
@@ -214,26 +268,27 @@ cudaError_t launch_csr_scatter(const int32_t* idx, int R, int E, const int32_t* 
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
   }
-  csr_scatter_kernel<<<nchunks, kCsrThreads, smem, stream>>>(idx, R, E, chunk_base, perm, inv);
+  csr_scatter_kernel<<<nchunks, kCsrThreads, smem, stream>>>(idx, R, E, chunk_base, perm, inv, mask, k);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, const int32_t* offsets, int E, int R, int k,
-                          int H, __nv_bfloat16* Xp, int* status, int num_sms, cudaStream_t stream) {
+                          int H, const float* scale, __nv_bfloat16* Xp, int* status, int num_sms,
+                          cudaStream_t stream) {
   if (R == 0) return cudaSuccess;
   const int rows_per_block = 8;
   const int blocks = static_cast<int>(std::min<int64_t>((R + rows_per_block - 1) / rows_per_block,
                                                         static_cast<int64_t>(num_sms) * 16));
-  gather_rows_kernel<<<blocks, 256, 0, stream>>>(x, perm, offsets, E, R, k, H, Xp, status);
+  gather_rows_kernel<<<blocks, 256, 0, stream>>>(x, perm, offsets, E, R, k, H, scale, Xp, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const __nv_bfloat16* Y, int T, int H, int k, __nv_bfloat16* out, int num_sms,
-                           cudaStream_t stream) {
+cudaError_t launch_combine(const __nv_bfloat16* Y, int T, int H, int k, const __nv_bfloat16* Ys, int Ns,
+                           const uint8_t* mask, __nv_bfloat16* out, int num_sms, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const int64_t n = static_cast<int64_t>(T) * (H / 8);
   const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(num_sms) * 16));
-  combine_kernel<<<blocks, 256, 0, stream>>>(Y, T, H, k, out);
+  combine_kernel<<<blocks, 256, 0, stream>>>(Y, T, H, k, Ys, Ns, mask, out);
   return cudaGetLastError();
 }
 

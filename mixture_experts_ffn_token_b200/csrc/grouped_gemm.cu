@@ -217,7 +217,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoo
         atomicOr(p.status, MOE_DEVICE_ERR_CSR);
       } else {
         dst = static_cast<int64_t>(slot) * p.H;
-        wgt = p.weights[slot];
+        wgt = p.weights != nullptr ? p.weights[slot] : 1.f;
       }
     } else {
       dst = (static_cast<int64_t>(tc.row0) + row) * p.D;

@@ -30,31 +30,37 @@ constexpr int kSmallWarps = 16;
 constexpr int kSmallSlots = 2048;
 constexpr int kSmallExperts = 512;
 cudaError_t launch_route_csr_small(const RouterArgs& a, int32_t* offsets, int32_t* perm, int* status,
-                                   cudaStream_t stream);
+                                   const uint8_t* mask, cudaStream_t stream);
 
 // ---------------------------------------------------------------------- CSR
 constexpr int kCsrChunk = 2048;      // slots per CTA
 constexpr int kCsrThreads = 512;     // 16 warps x 128 slots
 inline int csr_num_chunks(int64_t R) { return static_cast<int>((R + kCsrChunk - 1) / kCsrChunk); }
+// mask (may be null): slots of tokens whose mask byte is 0 take no place.
 cudaError_t launch_csr_count(const int32_t* idx, int R, int E, int32_t* chunk_counts, int* status,
-                             cudaStream_t stream);
+                             const uint8_t* mask, int k, cudaStream_t stream);
 cudaError_t launch_csr_scan(const int32_t* chunk_counts, int nchunks, int E, int32_t* chunk_base,
                             int32_t* offsets, cudaStream_t stream);
 cudaError_t launch_csr_scatter(const int32_t* idx, int R, int E, const int32_t* chunk_base, int32_t* perm,
-                               int32_t* inv, cudaStream_t stream);
+                               int32_t* inv, const uint8_t* mask, int k, cudaStream_t stream);
+cudaError_t launch_shared_index(int T, int Ns, int32_t* offsets, int32_t* perm, int num_sms, cudaStream_t stream);
 
 // ----------------------------------------------------- gather and combine
+// scale (may be null): per-slot factor applied to the gathered row.
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, const int32_t* offsets, int E, int R,
-                          int k, int H, __nv_bfloat16* Xp, int* status, int num_sms, cudaStream_t stream);
-cudaError_t launch_combine(const __nv_bfloat16* Y, int T, int H, int k, __nv_bfloat16* out, int num_sms,
-                           cudaStream_t stream);
+                          int k, int H, const float* scale, __nv_bfloat16* Xp, int* status, int num_sms,
+                          cudaStream_t stream);
+// Ys (may be null, Ns = 0): shared-expert rows added after the routed ones;
+// mask (may be null): masked tokens get zero rows.
+cudaError_t launch_combine(const __nv_bfloat16* Y, int T, int H, int k, const __nv_bfloat16* Ys, int Ns,
+                           const uint8_t* mask, __nv_bfloat16* out, int num_sms, cudaStream_t stream);
 
 // ------------------------------------------------------------ grouped GEMM
 struct GroupedGemmArgs {
   // routing (device)
   const int32_t* offsets;   // [E+1]
   const int32_t* perm;      // [R]
-  const float* weights;     // [R] routing weight per slot (down GEMM)
+  const float* weights;     // [R] routing weight per slot (down GEMM), or null for 1
   int E, R, T, k;
   // problem
   int H, D;

@@ -86,11 +86,25 @@ moe_status_t validate_config(const moe_config_t* c) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-struct WsLayout {
-  size_t status, chunk_counts, chunk_base, offsets, perm, idx, w, sink, xp, h, total;
+// The extensions of moe_forward_ex (token mask, router weight before the
+// experts, shared experts), already validated.
+struct Extras {
+  const uint8_t* mask = nullptr;
+  bool weight_first = false;
+  int Ns = 0, Ds = 0;
+  const void* s_gu_w = nullptr;
+  const void* s_gu_b = nullptr;
+  const void* s_d_w = nullptr;
+  const void* s_d_b = nullptr;
 };
 
-WsLayout ws_layout(const moe_config_t* c) {
+struct WsLayout {
+  size_t status, chunk_counts, chunk_base, offsets, perm, idx, w, sink, xp, h, total;
+  // shared experts: CSR of the [T, Ns] slot space, Xp_s (then Y_s), h_s
+  size_t sh_offsets = 0, sh_perm = 0, sh_x = 0, sh_h = 0;
+};
+
+WsLayout ws_layout(const moe_config_t* c, const Extras* ex = nullptr) {
   const size_t T = static_cast<size_t>(c->num_tokens), H = c->hidden_dim, E = c->num_experts, D = c->moe_dim;
   const size_t R = T * c->top_k;
   const size_t nchunks = static_cast<size_t>(moe::csr_num_chunks(static_cast<int64_t>(R)));
@@ -116,6 +130,17 @@ WsLayout ws_layout(const moe_config_t* c) {
   o += align256(R * H * 2);
   L.h = o;
   o += align256(R * D * 2);
+  if (ex != nullptr && ex->Ns > 0) {
+    const size_t Rs = T * static_cast<size_t>(ex->Ns);
+    L.sh_offsets = o;
+    o += align256((static_cast<size_t>(ex->Ns) + 1) * 4);
+    L.sh_perm = o;
+    o += align256(Rs * 4);
+    L.sh_x = o;  // Xp_s [T*Ns, H] for the shared gate_up GEMM, then Y_s
+    o += align256(Rs * H * 2);
+    L.sh_h = o;
+    o += align256(Rs * static_cast<size_t>(ex->Ds) * 2);
+  }
   L.total = o;
   return L;
 }
@@ -125,8 +150,9 @@ T* at(void* base, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(base) + off);
 }
 
-moe_status_t check_workspace(const moe_config_t* c, const void* ws, size_t bytes, WsLayout* L) {
-  *L = ws_layout(c);
+moe_status_t check_workspace(const moe_config_t* c, const void* ws, size_t bytes, WsLayout* L,
+                             const Extras* ex = nullptr) {
+  *L = ws_layout(c, ex);
   if (ws == nullptr || !aligned16(ws)) return MOE_ERR_INVALID_ARGUMENT;
   if (bytes < L->total) return MOE_ERR_WORKSPACE_TOO_SMALL;
   return MOE_OK;
@@ -160,24 +186,30 @@ moe::RouterArgs router_args(const moe_config_t* c, const void* logits, const flo
   return a;
 }
 
-// Gather -> gate_up GEMM -> down GEMM -> combine.  ev (may be null) gets a
-// record before each of the four kernels and after the last.
-moe_status_t enqueue_ffn(const moe_config_t* c, const void* x, const void* gate_up_w, const void* gate_up_b,
-                         const void* down_w, const void* down_b, const int32_t* offsets, const int32_t* perm,
-                         const float* weights, void* out, void* ws, const WsLayout& L, int num_sms,
-                         cudaStream_t stream, cudaEvent_t const* ev) {
-  const int T = c->num_tokens, H = c->hidden_dim, E = c->num_experts, k = c->top_k, D = c->moe_dim;
-  const int R = T * k;
-  int* status = at<int>(ws, L.status);
-  __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
-  __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
-  auto rec = [&](int i) {
+// Records ev[i] on the stream when events are requested.
+struct Recorder {
+  cudaEvent_t const* ev;
+  cudaStream_t stream;
+  void operator()(int i) const {
     if (ev != nullptr) cudaEventRecord(ev[i], stream);
-  };
-  rec(0);
-  cudaError_t err = moe::launch_gather(static_cast<const __nv_bfloat16*>(x), perm, offsets, E, R, k, H, xp, status,
-                                       num_sms, stream);
-  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  }
+};
+
+// One grouped expert FFN pass: gather (x rows by perm, times scale[slot] if
+// given) -> gate_up GEMM + activation -> down GEMM (+ bias, times
+// weights[slot] if given) writing Y at slot rows.  Y may alias xp (the
+// gate_up GEMM is done with it).  rec(base..base+2) before each kernel.
+moe_status_t enqueue_grouped_pass(const moe_config_t* c, int E, int k, int D, const void* x, const void* gate_up_w,
+                                  const void* gate_up_b, const void* down_w, const void* down_b,
+                                  const int32_t* offsets, const int32_t* perm, const float* scale,
+                                  const float* weights, __nv_bfloat16* xp, __nv_bfloat16* h, __nv_bfloat16* y,
+                                  int* status, int num_sms, cudaStream_t stream, const Recorder& rec, int base) {
+  const int T = c->num_tokens, H = c->hidden_dim;
+  const int R = T * k;
+  rec(base);
+  if (moe::launch_gather(static_cast<const __nv_bfloat16*>(x), perm, offsets, E, R, k, H, scale, xp, status,
+                         num_sms, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
   moe::GroupedGemmArgs g;
   g.offsets = offsets;
   g.perm = perm;
@@ -198,31 +230,45 @@ moe_status_t enqueue_ffn(const moe_config_t* c, const void* x, const void* gate_
   g.W = static_cast<const __nv_bfloat16*>(gate_up_w);
   g.bias = static_cast<const __nv_bfloat16*>(gate_up_b);
   g.out = h;
-  rec(1);
-  err = moe::launch_gemm_gate_up(g, stream);
-  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  rec(base + 1);
+  if (moe::launch_gemm_gate_up(g, stream) != cudaSuccess) return MOE_ERR_CUDA;
   g.A = h;
   g.W = static_cast<const __nv_bfloat16*>(down_w);
   g.bias = static_cast<const __nv_bfloat16*>(down_b);
-  g.out = xp;  // Y reuses the Xp region: the gate_up GEMM has finished with it
-  rec(2);
-  err = moe::launch_gemm_down(g, stream);
-  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  g.out = y;
+  rec(base + 2);
+  if (moe::launch_gemm_down(g, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+// Routed pass + combine (moe_grouped_ffn, and the tail of moe_forward
+// without extensions).  ev (may be null): before gather, gate_up GEMM, down
+// GEMM, combine, and after the combine.
+moe_status_t enqueue_ffn(const moe_config_t* c, const void* x, const void* gate_up_w, const void* gate_up_b,
+                         const void* down_w, const void* down_b, const int32_t* offsets, const int32_t* perm,
+                         const float* weights, void* out, void* ws, const WsLayout& L, int num_sms,
+                         cudaStream_t stream, cudaEvent_t const* ev) {
+  const Recorder rec{ev, stream};
+  __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
+  moe_status_t st = enqueue_grouped_pass(c, c->num_experts, c->top_k, c->moe_dim, x, gate_up_w, gate_up_b, down_w,
+                                         down_b, offsets, perm, nullptr, weights, xp, at<__nv_bfloat16>(ws, L.h),
+                                         xp, at<int>(ws, L.status), num_sms, stream, rec, 0);
+  if (st != MOE_OK) return st;
   rec(3);
-  err = moe::launch_combine(xp, T, H, k, static_cast<__nv_bfloat16*>(out), num_sms, stream);
-  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_combine(xp, c->num_tokens, c->hidden_dim, c->top_k, nullptr, 0, nullptr,
+                          static_cast<__nv_bfloat16*>(out), num_sms, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
   rec(4);
   return MOE_OK;
 }
 
 moe_status_t enqueue_csr(const moe_config_t* c, const int32_t* idx, int32_t* offsets, int32_t* perm, int32_t* inv,
-                         void* ws, const WsLayout& L, cudaStream_t stream, cudaEvent_t const* ev) {
-  const int R = c->num_tokens * c->top_k, E = c->num_experts;
-  auto rec = [&](int i) {
-    if (ev != nullptr) cudaEventRecord(ev[i], stream);
-  };
+                         void* ws, const WsLayout& L, cudaStream_t stream, cudaEvent_t const* ev,
+                         const uint8_t* mask = nullptr) {
+  const int R = c->num_tokens * c->top_k, E = c->num_experts, k = c->top_k;
+  const Recorder rec{ev, stream};
   rec(0);
-  if (moe::launch_csr_count(idx, R, E, at<int32_t>(ws, L.chunk_counts), at<int>(ws, L.status), stream) !=
+  if (moe::launch_csr_count(idx, R, E, at<int32_t>(ws, L.chunk_counts), at<int>(ws, L.status), mask, k, stream) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
   rec(1);
@@ -230,17 +276,54 @@ moe_status_t enqueue_csr(const moe_config_t* c, const int32_t* idx, int32_t* off
                            offsets, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   rec(2);
-  if (moe::launch_csr_scatter(idx, R, E, at<int32_t>(ws, L.chunk_base), perm, inv, stream) != cudaSuccess)
+  if (moe::launch_csr_scatter(idx, R, E, at<int32_t>(ws, L.chunk_base), perm, inv, mask, k, stream) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
-moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const void* logits, const float* expert_bias,
-                          const float* global_scale, const void* gate_up_w, const void* gate_up_b,
-                          const void* down_w, const void* down_b, void* out, int32_t* idx_out, float* w_out,
-                          float* sink_out, void* ws, size_t ws_bytes, cudaStream_t stream, cudaEvent_t const* ev) {
+// Host-side checks of moe_extras_t against the configuration.
+moe_status_t validate_extras(const moe_config_t* c, const moe_extras_t* e, Extras* out) {
+  *out = Extras{};
+  if (e == nullptr) return MOE_OK;
+  if (e->apply_router_weight_first != 0 && e->apply_router_weight_first != 1) return MOE_ERR_INVALID_ARGUMENT;
+  out->mask = e->token_mask;
+  out->weight_first = e->apply_router_weight_first == 1;
+  if (e->num_shared < 0) return MOE_ERR_INVALID_ARGUMENT;
+  if (e->num_shared == 0) return MOE_OK;
+  if (e->shared_dim <= 0) return MOE_ERR_INVALID_ARGUMENT;
+  if (e->shared_dim % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  // sink router: the sink lanes are the gates of the shared experts
+  if (c->router == MOE_ROUTER_SIGMOID_SINK && e->num_shared != c->num_sink) return MOE_ERR_INVALID_ARGUMENT;
+  if (e->num_shared > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(c->num_tokens) * e->num_shared > (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+  if (c->num_tokens > 0) {
+    if (e->shared_gate_up_w == nullptr || e->shared_down_w == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(e->shared_gate_up_w) || !aligned16(e->shared_down_w)) return MOE_ERR_INVALID_ARGUMENT;
+    if (check_bias(c, e->shared_gate_up_b, e->shared_down_b) != MOE_OK) return MOE_ERR_INVALID_ARGUMENT;
+  }
+  out->Ns = e->num_shared;
+  out->Ds = e->shared_dim;
+  out->s_gu_w = e->shared_gate_up_w;
+  out->s_gu_b = e->shared_gate_up_b;
+  out->s_d_w = e->shared_down_w;
+  out->s_d_b = e->shared_down_b;
+  return MOE_OK;
+}
+
+// moe_forward with or without extensions.  Event layouts: the plain timed
+// call records MOE_NUM_STAGE_EVENTS (router, 3 x CSR, gather, gate_up, down,
+// combine, end); with extensions MOE_NUM_STAGE_EVENTS_EX adds shared index,
+// shared gather, shared gate_up and shared down before the combine.
+moe_status_t forward_impl(const moe_config_t* cfg, const moe_extras_t* extras, const void* x, const void* logits,
+                          const float* expert_bias, const float* global_scale, const void* gate_up_w,
+                          const void* gate_up_b, const void* down_w, const void* down_b, void* out, int32_t* idx_out,
+                          float* w_out, float* sink_out, void* ws, size_t ws_bytes, cudaStream_t stream,
+                          cudaEvent_t const* ev) {
   moe_status_t st = validate_config(cfg);
   if (st != MOE_OK) return st;
+  Extras ex;
+  if ((st = validate_extras(cfg, extras, &ex)) != MOE_OK) return st;
   if (cfg->num_tokens == 0) return MOE_OK;  // nothing to read or write; empty tensors may have null pointers
   if (x == nullptr || logits == nullptr || gate_up_w == nullptr || down_w == nullptr || out == nullptr)
     return MOE_ERR_INVALID_ARGUMENT;
@@ -248,35 +331,66 @@ moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const void* lo
     return MOE_ERR_INVALID_ARGUMENT;
   if ((st = check_bias(cfg, gate_up_b, down_b)) != MOE_OK) return st;
   WsLayout L;
-  if ((st = check_workspace(cfg, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if ((st = check_workspace(cfg, ws, ws_bytes, &L, &ex)) != MOE_OK) return st;
   int num_sms = 0;
   if ((st = current_device(&num_sms)) != MOE_OK) return st;
+  const bool extended = extras != nullptr;
+  const Recorder rec{ev, stream};
+  const int T = cfg->num_tokens, k = cfg->top_k;
 
   int32_t* idx = idx_out != nullptr ? idx_out : at<int32_t>(ws, L.idx);
   float* w = w_out != nullptr ? w_out : at<float>(ws, L.w);
   float* sink = (sink_out != nullptr || cfg->num_sink == 0) ? sink_out : at<float>(ws, L.sink);
-  if (ev != nullptr) cudaEventRecord(ev[0], stream);
+  int* status = at<int>(ws, L.status);
+  rec(0);
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* perm = at<int32_t>(ws, L.perm);
-  const int64_t R = static_cast<int64_t>(cfg->num_tokens) * cfg->top_k;
+  const int64_t R = static_cast<int64_t>(T) * k;
   if (R <= moe::kSmallSlots && cfg->num_experts <= moe::kSmallExperts) {
     // small (decode-sized) problems: routing and the CSR build in one CTA;
     // the CSR stages then record back-to-back events
     const moe::RouterArgs ra = router_args(cfg, logits, expert_bias, global_scale, idx, w, sink, nullptr);
-    if (moe::launch_route_csr_small(ra, offsets, perm, at<int>(ws, L.status), stream) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    if (ev != nullptr)
-      for (int i = 1; i <= 3; ++i) cudaEventRecord(ev[i], stream);
+    if (moe::launch_route_csr_small(ra, offsets, perm, status, ex.mask, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    for (int i = 1; i <= 3; ++i) rec(i);
   } else {
-    const moe::RouterArgs ra =
-        router_args(cfg, logits, expert_bias, global_scale, idx, w, sink, at<int>(ws, L.status));
+    const moe::RouterArgs ra = router_args(cfg, logits, expert_bias, global_scale, idx, w, sink, status);
     if (moe::launch_router(ra, stream) != cudaSuccess) return MOE_ERR_CUDA;
-    if ((st = enqueue_csr(cfg, idx, offsets, perm, nullptr, ws, L, stream, ev != nullptr ? ev + 1 : nullptr)) !=
-        MOE_OK)
+    if ((st = enqueue_csr(cfg, idx, offsets, perm, nullptr, ws, L, stream, ev != nullptr ? ev + 1 : nullptr,
+                          ex.mask)) != MOE_OK)
       return st;
   }
-  return enqueue_ffn(cfg, x, gate_up_w, gate_up_b, down_w, down_b, offsets, perm, w, out, ws, L, num_sms, stream,
-                     ev != nullptr ? ev + 4 : nullptr);
+  if (!extended) return enqueue_ffn(cfg, x, gate_up_w, gate_up_b, down_w, down_b, offsets, perm, w, out, ws, L,
+                                    num_sms, stream, ev != nullptr ? ev + 4 : nullptr);
+
+  // routed pass: the weight scales the input (weight first) or the output
+  __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
+  st = enqueue_grouped_pass(cfg, cfg->num_experts, k, cfg->moe_dim, x, gate_up_w, gate_up_b, down_w, down_b, offsets,
+                            perm, ex.weight_first ? w : nullptr, ex.weight_first ? nullptr : w, xp,
+                            at<__nv_bfloat16>(ws, L.h), xp, status, num_sms, stream, rec, 4);
+  if (st != MOE_OK) return st;
+  __nv_bfloat16* ys = nullptr;
+  rec(7);
+  if (ex.Ns > 0) {
+    // shared experts: every token through each of them, gated by the sink
+    // weights (sink router) or by 1
+    int32_t* s_off = at<int32_t>(ws, L.sh_offsets);
+    int32_t* s_perm = at<int32_t>(ws, L.sh_perm);
+    if (moe::launch_shared_index(T, ex.Ns, s_off, s_perm, num_sms, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    const float* gates = cfg->router == MOE_ROUTER_SIGMOID_SINK ? sink : nullptr;
+    ys = at<__nv_bfloat16>(ws, L.sh_x);
+    st = enqueue_grouped_pass(cfg, ex.Ns, ex.Ns, ex.Ds, x, ex.s_gu_w, ex.s_gu_b, ex.s_d_w, ex.s_d_b, s_off, s_perm,
+                              ex.weight_first ? gates : nullptr, ex.weight_first ? nullptr : gates, ys,
+                              at<__nv_bfloat16>(ws, L.sh_h), ys, status, num_sms, stream, rec, 8);
+    if (st != MOE_OK) return st;
+  } else {
+    for (int i = 8; i <= 10; ++i) rec(i);
+  }
+  rec(11);
+  if (moe::launch_combine(xp, T, cfg->hidden_dim, k, ys, ex.Ns, ex.mask, static_cast<__nv_bfloat16*>(out), num_sms,
+                          stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  rec(12);
+  return MOE_OK;
 }
 
 }  // namespace
@@ -362,7 +476,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* log
                          const float* global_scale, const void* gate_up_w, const void* gate_up_b, const void* down_w,
                          const void* down_b, void* out, int32_t* expert_indices_out, float* expert_weights_out,
                          float* sink_weights_out, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
-  return forward_impl(cfg, x, logits, expert_bias, global_scale, gate_up_w, gate_up_b, down_w, down_b, out,
+  return forward_impl(cfg, nullptr, x, logits, expert_bias, global_scale, gate_up_w, gate_up_b, down_w, down_b, out,
                       expert_indices_out, expert_weights_out, sink_weights_out, workspace, workspace_bytes,
                       reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
@@ -375,9 +489,35 @@ moe_status_t moe_forward_timed(const moe_config_t* cfg, const void* x, const voi
   if (stage_events == nullptr) return MOE_ERR_INVALID_ARGUMENT;
   for (int i = 0; i < MOE_NUM_STAGE_EVENTS; ++i)
     if (stage_events[i] == nullptr) return MOE_ERR_INVALID_ARGUMENT;
-  return forward_impl(cfg, x, logits, expert_bias, global_scale, gate_up_w, gate_up_b, down_w, down_b, out,
+  return forward_impl(cfg, nullptr, x, logits, expert_bias, global_scale, gate_up_w, gate_up_b, down_w, down_b, out,
                       expert_indices_out, expert_weights_out, sink_weights_out, workspace, workspace_bytes,
                       reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<cudaEvent_t const*>(stage_events));
+}
+
+moe_status_t moe_workspace_size_ex(const moe_config_t* cfg, const moe_extras_t* extras, size_t* bytes) {
+  moe_status_t st = validate_config(cfg);
+  if (st != MOE_OK) return st;
+  Extras ex;
+  if ((st = validate_extras(cfg, extras, &ex)) != MOE_OK) return st;
+  if (bytes == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  *bytes = ws_layout(cfg, &ex).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_forward_ex(const moe_config_t* cfg, const moe_extras_t* extras, const void* x, const void* logits,
+                            const float* expert_bias, const float* global_scale, const void* gate_up_w,
+                            const void* gate_up_b, const void* down_w, const void* down_b, void* out,
+                            int32_t* expert_indices_out, float* expert_weights_out, float* sink_weights_out,
+                            void* workspace, size_t workspace_bytes, moe_stream_t stream, void* const* stage_events) {
+  if (stage_events != nullptr)
+    for (int i = 0; i < MOE_NUM_STAGE_EVENTS_EX; ++i)
+      if (stage_events[i] == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  moe_extras_t none;
+  std::memset(&none, 0, sizeof(none));
+  return forward_impl(cfg, extras != nullptr ? extras : &none, x, logits, expert_bias, global_scale, gate_up_w,
+                      gate_up_b, down_w, down_b, out, expert_indices_out, expert_weights_out, sink_weights_out,
+                      workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream),
+                      reinterpret_cast<cudaEvent_t const*>(stage_events));
 }
 
 moe_status_t moe_device_status(const void* workspace, int32_t* device_status, moe_stream_t stream) {

@@ -138,7 +138,8 @@ __global__ void __launch_bounds__(128) router_kernel(const RouterArgs a) {
 // and experts gives every slot its position, stable in slot order.
 template <int NPL, bool SINK, bool BF16>
 __global__ void __launch_bounds__(32 * kSmallWarps) route_csr_small_kernel(const RouterArgs a, int32_t* offsets,
-                                                                           int32_t* perm, int* status) {
+                                                                           int32_t* perm, int* status,
+                                                                           const uint8_t* mask) {
   extern __shared__ int sm[];
   int* s_idx = sm;                           // [R]
   int* wcnt = sm + kSmallSlots;              // [kSmallWarps][E]
@@ -149,7 +150,8 @@ __global__ void __launch_bounds__(32 * kSmallWarps) route_csr_small_kernel(const
   for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) wcnt[i] = 0;
   for (int t = warp; t < a.T; t += kSmallWarps) {
     const int e = route_token<NPL, SINK, BF16>(a, t, lane);
-    if (lane < a.k) s_idx[t * a.k + lane] = e;
+    // a masked token is routed (its weights are returned) but takes no slot
+    if (lane < a.k) s_idx[t * a.k + lane] = (mask == nullptr || mask[t] != 0) ? e : -2;
   }
   __syncthreads();
   constexpr int kPerWarp = kSmallSlots / kSmallWarps;
@@ -161,7 +163,7 @@ __global__ void __launch_bounds__(32 * kSmallWarps) route_csr_small_kernel(const
     const int s = wbase + r + lane;
     const int e = s < R ? s_idx[s] : -1;
     const bool ok = e >= 0 && e < E;
-    if (s < R && !ok) bad = true;
+    if (s < R && !ok && e != -2) bad = true;
     const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : E + lane);
     if (ok && (peers & lt_mask) == 0) my[e] += __popc(peers);
     __syncwarp();
@@ -236,15 +238,15 @@ cudaError_t launch_npl(const RouterArgs& a, cudaStream_t stream) {
 
 template <int NPL>
 cudaError_t launch_small_npl(const RouterArgs& a, int32_t* offsets, int32_t* perm, int* status,
-                             cudaStream_t stream) {
+                             const uint8_t* mask, cudaStream_t stream) {
   const size_t smem = (kSmallSlots + static_cast<size_t>(kSmallWarps) * a.E) * sizeof(int);
   const dim3 block(32 * kSmallWarps);
   if (a.sink) {
-    if (a.logits_bf16) route_csr_small_kernel<NPL, true, true><<<1, block, smem, stream>>>(a, offsets, perm, status);
-    else route_csr_small_kernel<NPL, true, false><<<1, block, smem, stream>>>(a, offsets, perm, status);
+    if (a.logits_bf16) route_csr_small_kernel<NPL, true, true><<<1, block, smem, stream>>>(a, offsets, perm, status, mask);
+    else route_csr_small_kernel<NPL, true, false><<<1, block, smem, stream>>>(a, offsets, perm, status, mask);
   } else {
-    if (a.logits_bf16) route_csr_small_kernel<NPL, false, true><<<1, block, smem, stream>>>(a, offsets, perm, status);
-    else route_csr_small_kernel<NPL, false, false><<<1, block, smem, stream>>>(a, offsets, perm, status);
+    if (a.logits_bf16) route_csr_small_kernel<NPL, false, true><<<1, block, smem, stream>>>(a, offsets, perm, status, mask);
+    else route_csr_small_kernel<NPL, false, false><<<1, block, smem, stream>>>(a, offsets, perm, status, mask);
   }
   return cudaGetLastError();
 }
@@ -252,13 +254,13 @@ cudaError_t launch_small_npl(const RouterArgs& a, int32_t* offsets, int32_t* per
 }  // namespace
 
 cudaError_t launch_route_csr_small(const RouterArgs& a, int32_t* offsets, int32_t* perm, int* status,
-                                   cudaStream_t stream) {
+                                   const uint8_t* mask, cudaStream_t stream) {
   const int per_lane = (a.E + 31) / 32;
-  if (per_lane <= 1) return launch_small_npl<1>(a, offsets, perm, status, stream);
-  if (per_lane <= 2) return launch_small_npl<2>(a, offsets, perm, status, stream);
-  if (per_lane <= 4) return launch_small_npl<4>(a, offsets, perm, status, stream);
-  if (per_lane <= 8) return launch_small_npl<8>(a, offsets, perm, status, stream);
-  return launch_small_npl<16>(a, offsets, perm, status, stream);
+  if (per_lane <= 1) return launch_small_npl<1>(a, offsets, perm, status, mask, stream);
+  if (per_lane <= 2) return launch_small_npl<2>(a, offsets, perm, status, mask, stream);
+  if (per_lane <= 4) return launch_small_npl<4>(a, offsets, perm, status, mask, stream);
+  if (per_lane <= 8) return launch_small_npl<8>(a, offsets, perm, status, mask, stream);
+  return launch_small_npl<16>(a, offsets, perm, status, mask, stream);
 }
 
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t stream) {

@@ -50,6 +50,15 @@ class Workload:
     global_scale: float = 1.0
     weight_std: float = 0.02
     bias_std: float = 0.01
+    # extensions (moe_forward_ex)
+    num_shared: int = 0               # shared experts (gated by the sink lanes under the sink router)
+    shared_dim: int = 0
+    weight_first: bool = False        # apply_router_weight_first
+    mask_frac: float = 0.0            # fraction of tokens masked out (token_mask)
+
+    @property
+    def extended(self) -> bool:
+        return self.num_shared > 0 or self.weight_first or self.mask_frac > 0
 
     @property
     def rows(self) -> int:
@@ -60,8 +69,9 @@ class Workload:
         return self.num_experts + self.num_sink
 
     def flops(self) -> int:
-        """Algorithmic FLOPs of the two grouped contractions: 2*R*H*2D + 2*R*D*H."""
-        return 6 * self.rows * self.hidden_dim * self.moe_dim
+        """Algorithmic FLOPs of the grouped contractions: 2*R*H*2D + 2*R*D*H,
+        plus the same for the T*Ns rows of the shared experts."""
+        return 6 * self.hidden_dim * (self.rows * self.moe_dim + self.num_tokens * self.num_shared * self.shared_dim)
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -77,6 +87,11 @@ WORKLOADS = {
     "decode": Workload("decode", 32, 4096, 64, 8, 1536, activation="gelu_tanh",
                        logits_kind="zipf_gumbel"),
 }
+# The sink-router workload with its two sink lanes as gated shared experts
+# (moe_dim-sized), and the Mixtral-shaped one with the router weight applied
+# before the experts: the two extension rows, measured by bench.py.
+WORKLOADS["sink_shared"] = WORKLOADS["sink"].replace(name="sink_shared", num_shared=2, shared_dim=768)
+WORKLOADS["mixtral_wfirst"] = WORKLOADS["mixtral"].replace(name="mixtral_wfirst", weight_first=True)
 
 
 def _normal(shape, std, gen, device, out_dtype=torch.bfloat16):
@@ -92,7 +107,9 @@ def make_inputs(wl: Workload, seed: int = 0, device: str | torch.device = "cpu",
 
     Returns a dict of tensors on `device`: x [T,H] bf16, logits [T,E+S] fp32,
     W_gu [E,H,2D] bf16, W_d [E,D,H] bf16, b_gu [E,2D] / b_d [E,H] bf16 or None,
-    expert_bias [E] fp32 or None, global_scale [1] fp32.
+    expert_bias [E] fp32 or None, global_scale [1] fp32, token_mask [T] uint8
+    or None, and with shared experts Ws_gu [Ns,H,2Ds], Ws_d [Ns,Ds,H] (and
+    bs_gu / bs_d with biases).
     """
     device = torch.device(device)
     gen = torch.Generator(device=device)
@@ -132,6 +149,19 @@ def make_inputs(wl: Workload, seed: int = 0, device: str | torch.device = "cpu",
             out["b_d"] = _normal((E, H), wl.bias_std, gen, device)
         else:
             out["b_gu"] = out["b_d"] = None
+        if wl.num_shared > 0:
+            Ns, Ds = wl.num_shared, wl.shared_dim
+            out["Ws_gu"] = _normal((Ns, H, 2 * Ds), wl.weight_std, gen, device)
+            out["Ws_d"] = _normal((Ns, Ds, H), wl.weight_std, gen, device)
+            if wl.has_bias:
+                out["bs_gu"] = _normal((Ns, 2 * Ds), wl.bias_std, gen, device)
+                out["bs_d"] = _normal((Ns, H), wl.bias_std, gen, device)
+            else:
+                out["bs_gu"] = out["bs_d"] = None
+    if wl.mask_frac > 0:
+        out["token_mask"] = (torch.rand(T, generator=gen, device=device) >= wl.mask_frac).to(torch.uint8)
+    else:
+        out["token_mask"] = None
     return out
 
 

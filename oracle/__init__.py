@@ -38,6 +38,9 @@ def _load():
         _lib.oracle_expert_ffn.restype = c_int
         _lib.oracle_expert_ffn.argtypes = [c_i64, c_int, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, vp,
                                            c_int, c_int, c_dbl, c_dbl, c_i64, vp, c_int, vp]
+        _lib.oracle_expert_ffn_ex.restype = c_int
+        _lib.oracle_expert_ffn_ex.argtypes = [c_i64, c_int, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, vp,
+                                              c_int, c_int, c_dbl, c_dbl, c_i64, vp, c_int, c_int, vp, vp]
         _lib.oracle_num_threads.restype = c_int
         _lib.oracle_num_threads.argtypes = []
     return _lib
@@ -117,7 +120,8 @@ def create_indices(idx, num_experts: int):
 
 
 def expert_ffn(x, idx, w, W_gu, W_d, b_gu=None, b_d=None, gate_up_format="concatenated",
-               activation="silu", alpha=0.0, limit=0.0, tokens=None, round_h_bf16=False):
+               activation="silu", alpha=0.0, limit=0.0, tokens=None, round_h_bf16=False,
+               weight_first=False, token_mask=None):
     """Grouped expert FFN in fp64.
 
     x [T,H], W_gu [E,H,2D], W_d [E,D,H], b_gu [E,2D], b_d [E,H]: bf16 bit
@@ -136,23 +140,51 @@ def expert_ffn(x, idx, w, W_gu, W_d, b_gu=None, b_d=None, gate_up_format="concat
     sel = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int64)
     n_out = T if sel is None else sel.size
     out = np.empty((n_out, H), np.float64)
-    rc = _load().oracle_expert_ffn(T, H, E, k, D, _ptr(x), _ptr(idx), _ptr(w), _ptr(_bits16(W_gu)),
-                                   _ptr(_bits16(b_gu)), _ptr(_bits16(W_d)), _ptr(_bits16(b_d)),
-                                   FORMAT_CODES[gate_up_format], ACT_CODES[activation], alpha, limit,
-                                   0 if sel is None else sel.size, _ptr(sel), int(bool(round_h_bf16)), _ptr(out))
+    mask = None if token_mask is None else np.ascontiguousarray(token_mask, dtype=np.uint8)
+    if mask is not None and mask.size != T:
+        raise ValueError("token_mask must have one byte per token")
+    rc = _load().oracle_expert_ffn_ex(T, H, E, k, D, _ptr(x), _ptr(idx), _ptr(w), _ptr(_bits16(W_gu)),
+                                      _ptr(_bits16(b_gu)), _ptr(_bits16(W_d)), _ptr(_bits16(b_d)),
+                                      FORMAT_CODES[gate_up_format], ACT_CODES[activation], alpha, limit,
+                                      0 if sel is None else sel.size, _ptr(sel), int(bool(round_h_bf16)),
+                                      int(bool(weight_first)), _ptr(mask), _ptr(out))
     if rc != 0:
         raise ValueError("oracle_expert_ffn: bad arguments")
     return out
 
 
+def shared_expert_ffn(x, gates, Ws_gu, Ws_d, bs_gu=None, bs_d=None, gate_up_format="concatenated",
+                      activation="silu", alpha=0.0, limit=0.0, tokens=None, weight_first=False, token_mask=None):
+    """Shared experts (StackedMoE has_shared_experts): every token goes through
+    all Ns of them; gates [T, Ns] weight them like routing weights (the sink
+    router's sink weights, or ones).  Evaluated as the routed FFN with every
+    token routed to experts 0..Ns-1."""
+    T = x.shape[0]
+    Ns = Ws_gu.shape[0]
+    idx = np.tile(np.arange(Ns, dtype=np.int32), (T, 1))
+    return expert_ffn(x, idx, gates, Ws_gu, Ws_d, bs_gu, bs_d, gate_up_format, activation, alpha, limit,
+                      tokens, weight_first=weight_first, token_mask=token_mask)
+
+
 def forward(x, logits, W_gu, W_d, b_gu=None, b_d=None, *, num_experts, top_k, router="softmax_topk",
             num_sink=0, expert_bias=None, route_scale=1.0, global_scale=1.0, gate_up_format="concatenated",
-            activation="silu", alpha=0.0, limit=0.0, tokens=None):
-    """Whole layer: router -> expert FFN.  Returns (out, idx, w, sink_w)."""
+            activation="silu", alpha=0.0, limit=0.0, tokens=None, weight_first=False, token_mask=None,
+            shared=None):
+    """Whole layer: router -> expert FFN (+ shared experts).  `shared` is None
+    or a dict with Ws_gu, Ws_d (and optional bs_gu, bs_d) of the shared
+    experts; their gates are the sink weights (sink router) or ones.
+    Returns (out, idx, w, sink_w)."""
     if router == "softmax_topk":
         idx, w = route_softmax_topk(logits, num_experts, top_k)
         sw = np.zeros((idx.shape[0], 0))
     else:
         idx, w, sw = route_sigmoid_sink(logits, num_experts, num_sink, top_k, expert_bias, route_scale, global_scale)
-    out = expert_ffn(x, idx, w, W_gu, W_d, b_gu, b_d, gate_up_format, activation, alpha, limit, tokens)
+    out = expert_ffn(x, idx, w, W_gu, W_d, b_gu, b_d, gate_up_format, activation, alpha, limit, tokens,
+                     weight_first=weight_first, token_mask=token_mask)
+    if shared is not None:
+        Ns = shared["Ws_gu"].shape[0]
+        gates = sw if router == "sigmoid_sink" else np.ones((idx.shape[0], Ns))
+        out = out + shared_expert_ffn(x, gates, shared["Ws_gu"], shared["Ws_d"], shared.get("bs_gu"),
+                                      shared.get("bs_d"), gate_up_format, activation, alpha, limit, tokens,
+                                      weight_first, token_mask)
     return out, idx, w, sw

@@ -40,6 +40,12 @@
 //       routing weight.
 //   R5  The CSR permutation lists flat slots t*k+j sorted by expert, stable
 //       (ascending slot inside one expert).
+//   R6  apply_router_weight_first (StackedMoE page): the weight scales the
+//       expert input, so the down bias is not weighted.  token_mask (NeMo
+//       GroupedExperts.forward): a masked token uses no expert and outputs a
+//       zero row.  Shared experts (StackedMoE has_shared_experts; the sink
+//       router page's "sink lanes are gated shared experts") are evaluated by
+//       the caller as this same FFN with every token routed to all of them.
 //
 // Inputs arrive as their stored bit patterns (bf16 as uint16, fp32 as float)
 // and are converted exactly to double; every operation after that is fp64.
@@ -214,10 +220,32 @@ int oracle_create_indices(int64_t R, int E, const int32_t* idx, int32_t* counts,
 // tokens_sel: NULL for every token (out is [T, H]) or n_sel token ids (out is
 // [n_sel, H] in that order).  round_h_bf16 != 0 rounds h to bf16 first (a
 // diagnostic, off for parity).  Returns 0, or -1 on bad arguments.
+int oracle_expert_ffn_ex(int64_t T, int H, int E, int k, int D, const uint16_t* x, const int32_t* idx,
+                         const double* w, const uint16_t* W_gu, const uint16_t* b_gu, const uint16_t* W_d,
+                         const uint16_t* b_d, int gate_up_format, int activation, double alpha, double limit,
+                         int64_t n_sel, const int64_t* tokens_sel, int round_h_bf16, int weight_first,
+                         const uint8_t* token_mask, double* out);
+
 int oracle_expert_ffn(int64_t T, int H, int E, int k, int D, const uint16_t* x, const int32_t* idx,
                       const double* w, const uint16_t* W_gu, const uint16_t* b_gu, const uint16_t* W_d,
                       const uint16_t* b_d, int gate_up_format, int activation, double alpha, double limit,
                       int64_t n_sel, const int64_t* tokens_sel, int round_h_bf16, double* out) {
+  return oracle_expert_ffn_ex(T, H, E, k, D, x, idx, w, W_gu, b_gu, W_d, b_d, gate_up_format, activation, alpha,
+                              limit, n_sel, tokens_sel, round_h_bf16, 0, nullptr, out);
+}
+
+// The same expert FFN with the two options of the layer pages:
+//   weight_first != 0 (StackedMoE apply_router_weight_first): the routing
+//     weight scales the expert's INPUT, out[t] = sum_j FFN_e(w[t,j] * x[t]),
+//     so the down bias is not weighted;
+//   token_mask (NeMo GroupedExperts.forward token_mask, NULL = all valid):
+//     a token whose mask byte is 0 goes through no expert and its output row
+//     is zero.
+int oracle_expert_ffn_ex(int64_t T, int H, int E, int k, int D, const uint16_t* x, const int32_t* idx,
+                         const double* w, const uint16_t* W_gu, const uint16_t* b_gu, const uint16_t* W_d,
+                         const uint16_t* b_d, int gate_up_format, int activation, double alpha, double limit,
+                         int64_t n_sel, const int64_t* tokens_sel, int round_h_bf16, int weight_first,
+                         const uint8_t* token_mask, double* out) {
   if (T < 0 || H < 1 || E < 1 || k < 1 || D < 1) return -1;
   const int64_t n_tok = tokens_sel ? n_sel : T;
   for (int64_t i = 0; i < n_tok; ++i) {
@@ -231,9 +259,10 @@ int oracle_expert_ffn(int64_t T, int H, int E, int k, int D, const uint16_t* x, 
   const int64_t N1 = 2 * static_cast<int64_t>(D);
 
   for (int e = 0; e < E; ++e) {
-    std::vector<int64_t> slots;  // local slot s = i*k + j, ascending
+    std::vector<int64_t> slots;  // local slot s = i*k + j, ascending; masked tokens take none
     for (int64_t s = 0; s < n_slots; ++s) {
       int64_t t = tokens_sel ? tokens_sel[s / k] : s / k;
+      if (token_mask && token_mask[t] == 0) continue;
       if (idx[t * k + s % k] == e) slots.push_back(s);
     }
     if (slots.empty()) continue;  // an expert with no tokens contributes nothing
@@ -245,8 +274,10 @@ int oracle_expert_ffn(int64_t T, int H, int E, int k, int D, const uint16_t* x, 
       const int64_t t = tokens_sel ? tokens_sel[s / k] : s / k;
       std::vector<double> a(N1, 0.0), h(D);
       for (int64_t n = 0; n < N1; ++n) a[n] = b_gu ? bf16_bits_to_double(b_gu[e * N1 + n]) : 0.0;
+      // the routing weight scales the input instead of the output
+      const double in_scale = weight_first ? w[t * k + s % k] : 1.0;
       for (int64_t c = 0; c < H; ++c) {
-        const double xc = bf16_bits_to_double(x[t * H + c]);
+        const double xc = in_scale * bf16_bits_to_double(x[t * H + c]);
         const uint16_t* row = Wg + c * N1;
         for (int64_t n = 0; n < N1; ++n) a[n] += xc * bf16_bits_to_double(row[n]);
       }
@@ -269,8 +300,8 @@ int oracle_expert_ffn(int64_t T, int H, int E, int k, int D, const uint16_t* x, 
     const int64_t t = tokens_sel ? tokens_sel[i] : i;
     double* o = out + i * H;
     for (int64_t c = 0; c < H; ++c) o[c] = 0.0;
-    for (int j = 0; j < k; ++j) {
-      const double wj = w[t * k + j];
+    for (int j = 0; j < k; ++j) {  // a masked token's slots were never computed: y is zero
+      const double wj = weight_first ? 1.0 : w[t * k + j];
       const double* ys = y.data() + (i * k + j) * H;
       for (int64_t c = 0; c < H; ++c) o[c] += wj * ys[c];
     }

@@ -88,3 +88,48 @@ def run_and_check(wl, seed=0, device_inputs=False, sample_tokens=None, out_guard
         guard = run.out_full[wl.num_tokens * wl.hidden_dim:].float()
         assert (guard == -7.0).all(), "output guard overwritten"
     return run, err
+
+
+def run_and_check_ex(wl, seed=0, device_inputs=False, sample_tokens=None):
+    """moe_forward_ex (mask / weight first / shared experts) against the oracle."""
+    inp = make_inputs(wl, seed, device="cuda" if device_inputs else "cpu")
+    d = to_dev(inp)
+    T, H, k, S = wl.num_tokens, wl.hidden_dim, wl.top_k, wl.num_sink
+    ex = abi.make_extras(token_mask=d["token_mask"], apply_router_weight_first=wl.weight_first,
+                         shared_gate_up_w=d.get("Ws_gu"), shared_down_w=d.get("Ws_d"),
+                         shared_gate_up_b=d.get("bs_gu"), shared_down_b=d.get("bs_d"))
+    cfg = abi.make_config(wl)
+    ws = torch.empty(abi.moe_workspace_size_ex(cfg, ex), dtype=torch.uint8, device="cuda")
+    out = torch.full((T, H), -7.0, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    sink = torch.empty((T, S), dtype=torch.float32, device="cuda") if S > 0 else None
+    abi.moe_forward_ex(cfg, ex, d["x"], d["logits"], d["W_gu"], d["W_d"], out, ws, gate_up_b=d["b_gu"],
+                       down_b=d["b_d"], expert_bias=d["expert_bias"], global_scale=d["global_scale"],
+                       expert_indices_out=idx, expert_weights_out=w, sink_weights_out=sink)
+    torch.cuda.synchronize()
+    assert abi.moe_device_status(ws) == 0
+    idx_ref, w_ref, s_ref = oracle_route(wl, inp)
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    check_weights(w.cpu().numpy(), w_ref)
+    tokens = None if sample_tokens is None else np.asarray(sample_tokens, dtype=np.int64)
+    mask = None if inp["token_mask"] is None else inp["token_mask"].cpu().numpy()
+    ref = oracle.expert_ffn(bf16_bits(inp["x"]), idx_ref, w_ref, bf16_bits(inp["W_gu"]), bf16_bits(inp["W_d"]),
+                            bf16_bits(inp["b_gu"]), bf16_bits(inp["b_d"]), wl.gate_up_format, wl.activation,
+                            wl.alpha, wl.limit, tokens=tokens, weight_first=wl.weight_first, token_mask=mask)
+    if wl.num_shared > 0:
+        gates = s_ref if wl.router == "sigmoid_sink" else np.ones((T, wl.num_shared))
+        ref = ref + oracle.shared_expert_ffn(bf16_bits(inp["x"]), gates, bf16_bits(inp["Ws_gu"]),
+                                             bf16_bits(inp["Ws_d"]), bf16_bits(inp.get("bs_gu")),
+                                             bf16_bits(inp.get("bs_d")), wl.gate_up_format, wl.activation,
+                                             wl.alpha, wl.limit, tokens=tokens, weight_first=wl.weight_first,
+                                             token_mask=mask)
+    got = out.float().cpu().numpy()
+    if tokens is not None:
+        got = got[tokens]
+    err = ffn_error(got, ref)
+    assert err <= FFN_TOL, f"ffn error {err:.3e} > {FFN_TOL}"
+    if mask is not None:
+        masked = (mask == 0) if tokens is None else (mask[tokens] == 0)
+        assert (got[masked] == 0).all(), "masked tokens must give zero rows"
+    return err

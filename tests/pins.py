@@ -377,5 +377,72 @@ def pin_ffn_empty_experts():
     assert np.isfinite(got).all() and np.array_equal(got, ref)
 
 
+def brute_force_weight_first(L, act, fmt, alpha=0.0, limit=0.0):
+    """Per-token loop: sum_j FFN_e(w_j * x[t]) with dense torch fp64 MLPs."""
+    T, k = L["idx"].shape
+    D = L["Wgu"].shape[2] // 2
+    out = torch.zeros(T, L["x"].shape[1], dtype=torch.float64)
+    for t in range(T):
+        for j in range(k):
+            e = int(L["idx"][t, j])
+            W = L["Wgu"][e].double()
+            Wg, Wu = (W[:, :D], W[:, D:]) if fmt == "concatenated" else (W[:, 0::2], W[:, 1::2])
+            bgu = None if L["bgu"] is None else L["bgu"][e].double()
+            bg, bu = (None, None) if bgu is None else ((bgu[:D], bgu[D:]) if fmt == "concatenated"
+                                                       else (bgu[0::2], bgu[1::2]))
+            bd = None if L["bd"] is None else L["bd"][e].double()
+            xin = float(L["w"][t, j]) * L["x"][t:t + 1].double()
+            out[t] += dense_ffn(xin, Wg, Wu, L["Wd"][e].double(), act, alpha, limit, bg, bu, bd)[0]
+    return out
+
+
+def pin_weight_first():
+    """apply_router_weight_first: the weight scales the input, so the down bias is unweighted."""
+    for fmt, act, alpha, limit, bias in (("concatenated", "silu", 0.0, 0.0, True),
+                                         ("interleaved", "swigluoai", ALPHA, LIMIT, True),
+                                         ("concatenated", "gelu_tanh", 0.0, 0.0, False)):
+        L = rand_layer(T=6, H=16, E=4, k=2, D=8, seed=23, bias=bias)
+        got = oracle.expert_ffn(L["xb"], L["idx"].numpy(), L["w"].numpy(), L["Wgub"], L["Wdb"], L["bgub"], L["bdb"],
+                                fmt, act, alpha, limit, weight_first=True)
+        ref = brute_force_weight_first(L, act, fmt, alpha, limit)
+        assert torch.allclose(torch.from_numpy(got), ref, rtol=1e-12, atol=1e-12), (fmt, act)
+    # with every weight 1 the two orders agree
+    L = rand_layer(T=5, H=16, E=4, k=2, D=8, seed=24, bias=True)
+    ones = np.ones((5, 2))
+    a = oracle.expert_ffn(L["xb"], L["idx"].numpy(), ones, L["Wgub"], L["Wdb"], L["bgub"], L["bdb"], weight_first=True)
+    b = oracle.expert_ffn(L["xb"], L["idx"].numpy(), ones, L["Wgub"], L["Wdb"], L["bgub"], L["bdb"])
+    assert np.array_equal(a, b)
+
+
+def pin_token_mask():
+    L = rand_layer(T=10, H=16, E=4, k=2, D=8, seed=25, bias=True)
+    mask = np.array([1, 0, 1, 1, 0, 0, 1, 1, 1, 0], np.uint8)
+    full = oracle.expert_ffn(L["xb"], L["idx"].numpy(), L["w"].numpy(), L["Wgub"], L["Wdb"], L["bgub"], L["bdb"])
+    got = oracle.expert_ffn(L["xb"], L["idx"].numpy(), L["w"].numpy(), L["Wgub"], L["Wdb"], L["bgub"], L["bdb"],
+                            token_mask=mask)
+    assert np.array_equal(got[mask == 1], full[mask == 1])       # valid tokens unchanged
+    assert (got[mask == 0] == 0).all()                           # masked tokens give zero rows
+    none = oracle.expert_ffn(L["xb"], L["idx"].numpy(), L["w"].numpy(), L["Wgub"], L["Wdb"], L["bgub"], L["bdb"],
+                             token_mask=np.zeros(10, np.uint8))
+    assert (none == 0).all()
+
+
+def pin_shared_experts():
+    """One shared expert with gate 1 adds one dense gated MLP (torch fp64)."""
+    g = torch.Generator().manual_seed(26)
+    T, H, Ds = 7, 24, 16
+    x, xb = bf16(torch.randn(T, H, generator=g))
+    Wgu, Wgub = bf16(torch.randn(1, H, 2 * Ds, generator=g) * 0.3)
+    Wd, Wdb = bf16(torch.randn(1, Ds, H, generator=g) * 0.3)
+    got = oracle.shared_expert_ffn(xb, np.ones((T, 1)), Wgub, Wdb, activation="silu")
+    ref = dense_ffn(x.double(), Wgu[0, :, :Ds].double(), Wgu[0, :, Ds:].double(), Wd[0].double(), "silu")
+    assert torch.allclose(torch.from_numpy(got), ref, rtol=1e-12, atol=1e-12)
+    # gates scale the shared outputs (sink lanes are gated shared experts)
+    gates = np.linspace(0.1, 1.3, T).reshape(T, 1)
+    got = oracle.shared_expert_ffn(xb, gates, Wgub, Wdb, activation="silu")
+    assert torch.allclose(torch.from_numpy(got), ref * torch.from_numpy(gates), rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [pin_activation_closed_forms, pin_activation_library_routines, pin_softmax_router, pin_sink_router,
-            pin_csr, pin_ffn_dense_reduction, pin_ffn_brute_force, pin_ffn_invariants, pin_ffn_empty_experts]
+            pin_csr, pin_ffn_dense_reduction, pin_ffn_brute_force, pin_ffn_invariants, pin_ffn_empty_experts,
+            pin_weight_first, pin_token_mask, pin_shared_experts]

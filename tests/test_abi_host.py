@@ -130,3 +130,35 @@ def test_zero_tokens_is_a_no_op(lib):
     # returns before any device call: nothing to do
     assert lib.moe_forward(ctypes.byref(cfg), FAKE, FAKE, None, None, FAKE, None, FAKE, None, FAKE, None, None,
                            None, FAKE, need, None) == 0
+
+
+def test_extras_validation(lib):
+    by = ctypes.byref
+    n = ctypes.c_size_t(0)
+    cfg = cfg_for("tiny")
+    base = abi.moe_workspace_size(cfg)
+    assert lib.moe_workspace_size_ex(by(cfg), None, by(n)) == 0 and n.value == base
+    ex = abi.MoEExtras()
+    ex.num_shared, ex.shared_dim = 2, 64
+    ex.shared_gate_up_w = ex.shared_down_w = FAKE
+    assert lib.moe_workspace_size_ex(by(cfg), by(ex), by(n)) == 0 and n.value > base
+    ex.shared_dim = 12
+    assert lib.moe_workspace_size_ex(by(cfg), by(ex), by(n)) == UNSUPPORTED
+    ex.shared_dim = 0
+    assert lib.moe_workspace_size_ex(by(cfg), by(ex), by(n)) == INVALID
+    ex = abi.MoEExtras()
+    ex.apply_router_weight_first = 2
+    assert lib.moe_workspace_size_ex(by(cfg), by(ex), by(n)) == INVALID
+    # the sink router gates its shared experts with the sink lanes: counts must agree
+    scfg = cfg_for("sink")
+    ex = abi.MoEExtras()
+    ex.num_shared, ex.shared_dim = 1, 64
+    ex.shared_gate_up_w = ex.shared_down_w = FAKE
+    assert lib.moe_workspace_size_ex(by(scfg), by(ex), by(n)) == INVALID
+    ex.num_shared = 2
+    assert lib.moe_workspace_size_ex(by(scfg), by(ex), by(n)) == 0
+    # shared experts need their weights
+    ex.shared_down_w = None
+    need = abi.moe_workspace_size(scfg)
+    assert lib.moe_forward_ex(by(scfg), by(ex), FAKE, FAKE, None, None, FAKE, None, FAKE, None, FAKE, None, None,
+                              None, FAKE, need * 4, None, None) == INVALID

@@ -1,0 +1,68 @@
+"""moe_forward_ex -- token mask, router weight before the experts, shared
+experts gated by the sink lanes (or ungated) -- against the fp64 oracle on
+seeded inputs; same bars as the core path."""
+import math
+
+import pytest
+import torch
+
+from gpu_helpers import GpuRun, run_and_check_ex, to_dev
+from mixture_experts_ffn_token_b200 import abi
+from mixture_experts_ffn_token_b200.workloads import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+MIX = WORKLOADS["mixtral"].replace(num_tokens=256, hidden_dim=512, moe_dim=384, logits_std=0.02 * math.sqrt(512))
+GPT = WORKLOADS["gptoss"].replace(num_tokens=96, hidden_dim=328, num_experts=16, moe_dim=200)
+SNK = WORKLOADS["sink"].replace(num_tokens=300, hidden_dim=256, num_experts=32, moe_dim=136)
+DEC = WORKLOADS["decode"].replace(num_tokens=8, hidden_dim=512, num_experts=16, moe_dim=192)
+
+
+@pytest.mark.parametrize("wl", [MIX, GPT, DEC, SNK.replace(num_tokens=1200)], ids=["mix", "gpt", "dec", "snk_big"])
+def test_weight_first(wl):
+    run_and_check_ex(wl.replace(weight_first=True), seed=1)
+
+
+@pytest.mark.parametrize("wl", [MIX, SNK, SNK.replace(num_tokens=1200), WORKLOADS["tiny"]],
+                         ids=["mix", "snk", "snk_big", "tiny"])
+def test_token_mask(wl):
+    run_and_check_ex(wl.replace(mask_frac=0.3), seed=2)
+
+
+@pytest.mark.parametrize("wl", [SNK.replace(num_shared=2, shared_dim=136),
+                                MIX.replace(num_shared=1, shared_dim=256),
+                                GPT.replace(num_shared=1, shared_dim=96),
+                                SNK.replace(num_tokens=1200, num_shared=2, shared_dim=72)],
+                         ids=["sink_gated", "softmax_ungated", "gpt_bias", "sink_big"])
+def test_shared_experts(wl):
+    run_and_check_ex(wl, seed=3)
+
+
+def test_everything_together():
+    run_and_check_ex(SNK.replace(num_shared=2, shared_dim=136, weight_first=True, mask_frac=0.25), seed=4)
+    run_and_check_ex(GPT.replace(num_shared=1, shared_dim=200, weight_first=True, mask_frac=0.5), seed=5)
+
+
+def test_no_extras_equals_forward():
+    """moe_forward_ex with no extensions gives moe_forward's output bit for bit."""
+    wl = SNK.replace(num_tokens=1200)
+    d = to_dev(make_inputs(wl, 6))
+    run = GpuRun(wl, d)
+    out = torch.empty_like(run.out)
+    sink = torch.empty_like(run.sink)
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(abi.NUM_STAGE_EVENTS_EX)]
+    abi.moe_forward_ex(run.cfg, None, d["x"], d["logits"], d["W_gu"], d["W_d"], out, run.ws,
+                       expert_bias=d["expert_bias"], global_scale=d["global_scale"], sink_weights_out=sink,
+                       events=events)
+    torch.cuda.synchronize()
+    assert torch.equal(out, run.out) and torch.equal(sink, run.sink)
+    assert sum(events[i].elapsed_time(events[i + 1]) for i in range(abi.NUM_STAGE_EVENTS_EX - 1)) > 0
+
+
+@pytest.mark.parametrize("name", ["sink_shared", "mixtral_wfirst"])
+def test_extension_workloads_full_size_sampled(name):
+    import numpy as np
+    wl = WORKLOADS[name]
+    rng = np.random.default_rng(7)
+    sample = np.unique(np.concatenate([[0, wl.num_tokens - 1], rng.choice(wl.num_tokens, 10, replace=False)]))
+    run_and_check_ex(wl, seed=0, device_inputs=True, sample_tokens=sample)

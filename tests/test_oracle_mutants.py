@@ -33,6 +33,11 @@ MUTANTS = {
     "up_clamp_sign": ("u = std::min(std::max(u, -limit), limit);\n      }\n      return g / (1.0",
                       "u = std::min(std::max(u, limit), limit);\n      }\n      return g / (1.0"),
     "swigluoai_alpha_ignored": ("std::exp(-alpha * g)", "std::exp(-g)"),
+    "weight_first_ignored": ("const double in_scale = weight_first ? w[t * k + s % k] : 1.0;",
+                             "const double in_scale = 1.0;"),
+    "weight_first_also_weights_output": ("const double wj = weight_first ? 1.0 : w[t * k + j];",
+                                         "const double wj = w[t * k + j];"),
+    "mask_ignored": ("      if (token_mask && token_mask[t] == 0) continue;\n", ""),
 }
 
 
@@ -56,7 +61,7 @@ def test_mutant_is_caught(name, source, tmp_path):
     import ctypes
     mutant = ctypes.CDLL(str(lib))
     for fn in ("oracle_activation", "oracle_route_softmax_topk", "oracle_route_sigmoid_sink",
-               "oracle_create_indices", "oracle_expert_ffn", "oracle_num_threads"):
+               "oracle_create_indices", "oracle_expert_ffn", "oracle_expert_ffn_ex", "oracle_num_threads"):
         getattr(mutant, fn).restype = getattr(real, fn).restype
         getattr(mutant, fn).argtypes = getattr(real, fn).argtypes
     caught = []
