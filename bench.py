@@ -56,12 +56,14 @@ def max_over_ranks(x, dist_mod, device):
     return float(t.item())
 
 
-def launches_per_step(wl):
+def launches_per_step(wl, single_launch):
     """Kernels one call launches: router + 3-kernel CSR build (one kernel
-    when T*k <= 2048 and E <= 512), gather, two grouped GEMMs, combine, and
-    with shared experts their index, gather and two GEMMs."""
+    when T*k <= 2048 and E <= 512), gather, the two grouped GEMMs (one
+    launch when fused), combine, and with shared experts their index,
+    gather and GEMMs."""
     small = wl.num_tokens * wl.top_k <= 2048 and wl.num_experts <= 512
-    return (1 if small else 4) + 3 + (4 if wl.num_shared > 0 else 0) + 1
+    gemms = 1 if single_launch else 2
+    return (1 if small else 4) + 1 + gemms + ((2 + gemms) if wl.num_shared > 0 else 0) + 1
 
 
 def job_throughput(world, tokens_per_rank, ms_per_step):
@@ -472,11 +474,14 @@ def run_gpu(args, wl):
     out_bytes = T * H * 2
 
     # ---------------- roofline of the dominant kernel
-    names = abi.STAGE_NAMES_EX if extras is not None else abi.STAGE_NAMES
+    names = list(abi.STAGE_NAMES_EX if extras is not None else abi.STAGE_NAMES)
+    fused = abi.moe_single_launch_ffn()
+    if fused:
+        # the "gate_up" stage is the single launch of both GEMMs; "down" is empty
+        names = [{"gemm_gate_up": "mega_ffn", "gemm_down": "(fused)", "shared_gemm_gate_up": "shared_mega_ffn",
+                  "shared_gemm_down": "(shared fused)"}.get(n, n) for n in names]
     flops = wl.flops()
     wbytes, used = touched_expert_bytes(wl, idx)
-    gate_up_flops = 4 * T * k * H * wl.moe_dim
-    down_flops = 2 * T * k * H * wl.moe_dim
     shared_rows = T * wl.num_shared
     dom = max(range(len(names)), key=lambda i: stage_ms[i])
     dom_name = names[dom]
@@ -486,14 +491,17 @@ def run_gpu(args, wl):
     capped = "sw_power_cap" in clock_summary.get("reasons", [])
     bf16_peak = peaks.get("bf16_tflops_sustained" if capped else "bf16_tflops", peaks.get("bf16_tflops"))
     bf16_kind = "sustained" if capped else "burst"
-    if dom_name in ("gemm_gate_up", "gemm_down", "shared_gemm_gate_up", "shared_gemm_down"):
-        up = dom_name.endswith("gate_up")
+    gemm_stages = ("gemm_gate_up", "gemm_down", "shared_gemm_gate_up", "shared_gemm_down", "mega_ffn",
+                   "shared_mega_ffn")
+    if dom_name in gemm_stages:
+        # FLOP / weight-byte multipliers: gate_up 4 / 2, down 2 / 1, both 6 / 3
+        fm, bm = (6, 3) if dom_name.endswith("mega_ffn") else (4, 2) if dom_name.endswith("gate_up") else (2, 1)
         if dom_name.startswith("shared"):
-            kflops = (4 if up else 2) * shared_rows * H * wl.shared_dim
-            kbytes = (2 if up else 1) * wl.num_shared * H * wl.shared_dim * 2
+            kflops = fm * shared_rows * H * wl.shared_dim
+            kbytes = bm * wl.num_shared * H * wl.shared_dim * 2
         else:
-            kflops = gate_up_flops if up else down_flops
-            kbytes = (2 if up else 1) * used * H * wl.moe_dim * 2
+            kflops = fm * T * k * H * wl.moe_dim
+            kbytes = bm * used * H * wl.moe_dim * 2
         t_flop = kflops / (bf16_peak * 1e12)
         t_byte = kbytes / (peaks["hbm_gbs"] * 1e9)
         if t_flop >= t_byte:
@@ -526,7 +534,8 @@ def run_gpu(args, wl):
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x_h_bytes,
                 "d2h_bytes_per_step": out_bytes},
-        "gpu_launches": launches_per_step(wl) * args.steps,
+        "gpu_launches": launches_per_step(wl, fused) * args.steps,
+        "single_launch_ffn": fused,
         "clocks": clock_summary,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -114,6 +114,7 @@ typedef struct {
 #define MOE_DEVICE_ERR_CSR            0x2  /* offsets not a CSR of R slots, or a permutation entry out of range */
 #define MOE_DEVICE_ERR_TIMEOUT_GEMM1  0x4  /* a gate_up GEMM pipeline wait gave up */
 #define MOE_DEVICE_ERR_TIMEOUT_GEMM2  0x8  /* a down GEMM pipeline wait gave up */
+/* (a wait that gives up inside the single-launch FFN sets both GEMM bits) */
 
 /* Number of events moe_forward_timed() records (one before each stage and
  * one after the last). */
@@ -123,8 +124,9 @@ const char* moe_status_string(moe_status_t status);
 
 /* Bytes of device workspace that any call below needs for this
  * configuration.  Host only, no CUDA calls.  The workspace holds the device
- * status word, the CSR scratch, the gathered rows Xp [R,H] (reused for the
- * unreduced expert outputs Y [R,H]) and the activations h [R,D], all bf16. */
+ * status word, the CSR scratch, the gathered rows Xp [R,H], the activations
+ * h [R,D] and the unreduced expert outputs Y [R,H] (bf16), and the
+ * single-launch FFN's per-piece arrival counters. */
 moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes);
 
 /* Stage 1, the router (sink_gate_router_kernel page, Args; softmax top-k
@@ -157,7 +159,13 @@ moe_status_t moe_create_indices(const moe_config_t* cfg, const int32_t* expert_i
 
 /* Stages 3 and 4 given a routing: gather the routed rows, grouped gate_up GEMM
  * + bias + activation (tcgen05 tensor cores), grouped down GEMM + bias, times
- * the routing weight, and the per-token sum over the k slots.
+ * the routing weight, and the per-token sum over the k slots.  By default
+ * the two GEMMs run as ONE persistent cooperative launch (the MegaFFN page's
+ * single launch: a down tile of a 128-row piece starts as soon as every
+ * gate_up tile of that piece has stored its h, signalled through per-piece
+ * arrival counters in the workspace, every wait bounded); the environment
+ * variable MOE_B200_SINGLE_LAUNCH=0 selects two launches instead (same
+ * results bit for bit; see moe_single_launch_ffn).
  *   x              [T, H] bf16.
  *   gate_up_w      [E, H, 2D] bf16 (StackedMoE gate_up_proj layout).
  *   gate_up_b      [E, 2D] bf16 or NULL (per has_bias).
@@ -179,8 +187,9 @@ moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x, const void*
  * the routing kept in the workspace.  expert_indices_out [T,k],
  * expert_weights_out [T,k] and sink_weights_out [T,S] are optional copies of
  * the routing (NULL = not returned; sink_weights_out is written only when
- * S > 0).  Eight kernel launches (five when T*k <= 2048 and E <= 512: the
- * router and the CSR build then share one single-CTA kernel), no host
+ * S > 0).  Seven kernel launches (four when T*k <= 2048 and E <= 512: the
+ * router and the CSR build then share one single-CTA kernel; one more each
+ * with MOE_B200_SINGLE_LAUNCH=0), no host
  * synchronisation, no allocation, so the call can be captured in a CUDA
  * graph. */
 moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* logits,
@@ -193,7 +202,13 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* log
  * (cudaEvent_t handles created by the caller) on `stream` before router,
  * CSR count, CSR scan, CSR scatter, gather, gate_up GEMM, down GEMM and
  * combine, and after the combine, so a caller can time each kernel on the
- * stream it runs on. */
+ * stream it runs on.  With the single-launch FFN the "gate_up GEMM" stage
+ * is the fused launch and the "down GEMM" stage is empty. */
+/* *enabled = 1 if moe_grouped_ffn / moe_forward / moe_forward_ex called now
+ * in this process run the two GEMMs as one launch, 0 if as two (the
+ * MOE_B200_SINGLE_LAUNCH setting, read at each call). */
+moe_status_t moe_single_launch_ffn(int32_t* enabled);
+
 moe_status_t moe_forward_timed(const moe_config_t* cfg, const void* x, const void* logits,
                                const float* expert_bias, const float* global_scale, const void* gate_up_w,
                                const void* gate_up_b, const void* down_w, const void* down_b, void* out,

@@ -32,7 +32,7 @@ STAGE_NAMES = ("router", "csr_count", "csr_scan", "csr_scatter", "gather", "gemm
 
 EXPORTED = ("moe_status_string", "moe_workspace_size", "moe_route", "moe_create_indices", "moe_grouped_ffn",
             "moe_forward", "moe_forward_timed", "moe_device_status", "moe_create_indices_noalloc",
-            "moe_workspace_size_ex", "moe_forward_ex")
+            "moe_workspace_size_ex", "moe_forward_ex", "moe_single_launch_ffn")
 NUM_STAGE_EVENTS_EX = 13
 STAGE_NAMES_EX = ("router", "csr_count", "csr_scan", "csr_scatter", "gather", "gemm_gate_up", "gemm_down",
                   "shared_index", "shared_gather", "shared_gemm_gate_up", "shared_gemm_down", "combine")
@@ -130,6 +130,8 @@ def load_library():
     lib.moe_workspace_size_ex.argtypes = [cfgp, exp, ctypes.POINTER(ctypes.c_size_t)]
     lib.moe_forward_ex.restype = ctypes.c_int
     lib.moe_forward_ex.argtypes = [cfgp, exp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+    lib.moe_single_launch_ffn.restype = ctypes.c_int
+    lib.moe_single_launch_ffn.argtypes = [ctypes.POINTER(ctypes.c_int32)]
     _lib = lib
     return lib
 
@@ -234,6 +236,14 @@ def moe_forward_timed(cfg, events, x, logits, gate_up_w, down_w, out, workspace,
                                             _p(out), _p(expert_indices_out), _p(expert_weights_out),
                                             _p(sink_weights_out), _p(workspace), workspace.numel(),
                                             _stream(stream), arr), "moe_forward_timed")
+
+
+def moe_single_launch_ffn() -> bool:
+    """Whether the two grouped GEMMs run as one launch in this process (set
+    MOE_B200_SINGLE_LAUNCH=0 in the environment for two launches)."""
+    v = ctypes.c_int32(0)
+    _check(load_library().moe_single_launch_ffn(ctypes.byref(v)), "moe_single_launch_ffn")
+    return bool(v.value)
 
 
 def moe_workspace_size_ex(cfg: MoEConfig, extras: Optional[MoEExtras]) -> int:

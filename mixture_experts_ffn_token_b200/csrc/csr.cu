@@ -151,7 +151,11 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
                                                           const int32_t* __restrict__ perm,
                                                           const int32_t* __restrict__ offsets, int E, int R, int k,
                                                           int H, const float* __restrict__ scale,
-                                                          __nv_bfloat16* __restrict__ Xp, int* status) {
+                                                          __nv_bfloat16* __restrict__ Xp, int* status,
+                                                          int* __restrict__ zero, int n_zero) {
+  // Clear the caller's counters (the single-launch FFN's per-piece arrival
+  // counts) for the kernel that follows on the stream.
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_zero; i += gridDim.x * blockDim.x) zero[i] = 0;
   int total = offsets[E];
   if (total < 0 || total > R) {
     if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, MOE_DEVICE_ERR_CSR);
@@ -274,12 +278,12 @@ cudaError_t launch_csr_scatter(const int32_t* idx, int R, int E, const int32_t* 
 
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, const int32_t* offsets, int E, int R, int k,
                           int H, const float* scale, __nv_bfloat16* Xp, int* status, int num_sms,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, int* zero, int n_zero) {
   if (R == 0) return cudaSuccess;
   const int rows_per_block = 8;
   const int blocks = static_cast<int>(std::min<int64_t>((R + rows_per_block - 1) / rows_per_block,
                                                         static_cast<int64_t>(num_sms) * 16));
-  gather_rows_kernel<<<blocks, 256, 0, stream>>>(x, perm, offsets, E, R, k, H, scale, Xp, status);
+  gather_rows_kernel<<<blocks, 256, 0, stream>>>(x, perm, offsets, E, R, k, H, scale, Xp, status, zero, n_zero);
   return cudaGetLastError();
 }
 

@@ -91,7 +91,7 @@ struct GemmParams {
 };
 
 struct TileCoord {
-  int e, row0, rows, n;
+  int e, row0, rows, n, piece;  // piece: global index of the 128-row piece
 };
 
 // Tile t -> (expert, first permuted row of the tile, valid rows, output
@@ -113,12 +113,52 @@ __device__ __forceinline__ TileCoord decode_tile(int t, int n_tiles, int E, cons
   const int m = local - c.n * mt;
   c.row0 = s_off[lo] + m * piece;
   c.rows = min(piece, s_off[lo + 1] - c.row0);
+  c.piece = s_mt[lo] + m;
   return c;
 }
 
 __device__ __forceinline__ bool wait_time_only(uint32_t bar, uint32_t parity) {
   int never = 0;
   return mbar_wait(bar, parity, &never, kTimeoutNs);
+}
+
+// ------------------------------------------ single-launch cross-CTA hand-off
+// A gate_up tile's epilogue warps each publish their h stores with one
+// release add on the piece's arrival counter; the producer of a down tile
+// waits (acquire) until all of the piece's gate_up tiles have arrived, then
+// orders those generic-proxy stores before its TMA (async-proxy) reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_release_add(int* addr, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire(const int* addr) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+  return v;
+}
+
+// Bounded wait for *counter >= target.  Gives up (false, CTA abort raised,
+// err bits recorded at once so other CTAs stop waiting too) after the
+// timeout, when this CTA aborts, or when another CTA has recorded a timeout.
+__device__ __forceinline__ bool wait_arrivals(const int* counter, int target, volatile int* abort,
+                                              volatile int* status, int err_bits) {
+  if (ld_acquire(counter) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1; it < (1u << 26); ++it) {
+    __nanosleep(64);
+    if (ld_acquire(counter) >= target) return true;
+    if ((it & 15u) == 0) {
+      if (*abort || (*status & err_bits) != 0) break;
+      if (global_timer_ns() - t0 > kTimeoutNs) break;
+    }
+  }
+  *abort = 1;
+  atomicOr(const_cast<int*>(status), err_bits);
+  return false;
 }
 
 // ----------------------------------------------------------- epilogues
@@ -261,10 +301,19 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoo
 }
 
 // ------------------------------------------------------------- the kernel
-template <int MODE, int PAIR>
+// FUSED = false: one contraction (MODE) over its tile list.  FUSED = true
+// (single-CTA tiles only): the gate_up contraction (MODE, maps A/B, params p)
+// followed in the same tile list by the down contraction (maps A2/B2, params
+// p2); tile t < total1 is a gate_up tile, the rest are down tiles, and every
+// CTA walks the list in increasing order, so a down tile only ever waits on
+// gate_up tiles that precede it and that some resident CTA has already
+// started (the launch is cooperative: all CTAs are resident).
+template <int MODE, int PAIR, bool FUSED>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                        const GemmParams p) {
+                        const __grid_constant__ CUtensorMap mapA2, const __grid_constant__ CUtensorMap mapB2,
+                        const GemmParams p, const GemmParams p2, int* arrivals) {
+  static_assert(!FUSED || (PAIR == 1 && MODE != MODE_DOWN), "the fused form is gate_up then down, one CTA a tile");
   using G = Geo<PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -305,6 +354,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fence_mbar_init();
     tma_prefetch_map(&mapA);
     tma_prefetch_map(&mapB);
+    if constexpr (FUSED) {
+      tma_prefetch_map(&mapA2);
+      tma_prefetch_map(&mapB2);
+    }
   }
   if (warp == 1) {
     if constexpr (PAIR == 2) {
@@ -354,9 +407,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
   const bool bad = *bad_flag != 0;
   if (bad && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.status, MOE_DEVICE_ERR_CSR);
-  const int total_tiles = bad ? 0 : s_mt[p.E] * p.n_tiles;
+  const int total1 = bad ? 0 : s_mt[p.E] * p.n_tiles;
+  const int total_tiles = total1 + (FUSED && !bad ? s_mt[p.E] * p2.n_tiles : 0);
   const int first_tile = blockIdx.x / PAIR;
   const int tile_stride = gridDim.x / PAIR;
+  // down tiles of a piece wait for this many arrivals (one per epilogue warp
+  // of each of the piece's gate_up tiles)
+  const int arrivals_needed = NUM_EPI_WARPS * p.n_tiles;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -364,9 +421,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int it = 0;
       bool ok = true;
       for (int t = first_tile; ok && t < total_tiles; t += tile_stride) {
-        const TileCoord tc = decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
+        const bool ph2 = FUSED && t >= total1;
+        const TileCoord tc = ph2 ? decode_tile(t - total1, p2.n_tiles, p.E, s_mt, s_off, G::PIECE)
+                                 : decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
         const int arow = tc.row0 + static_cast<int>(rank) * BM;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        const int nkb = ph2 ? p2.num_kb : p.num_kb;
+        if constexpr (FUSED) {
+          if (ph2) {
+            if (!wait_arrivals(arrivals + tc.piece, arrivals_needed, abort_flag, p.status, p.err_bit)) {
+              ok = false;
+              break;
+            }
+            fence_proxy_async_global();  // h stores (generic proxy) before the TMA reads of h
+          }
+        }
+        for (int kb = 0; kb < nkb; ++kb) {
           const int s = it % G::STAGES;
           const uint32_t ph = static_cast<uint32_t>(it / G::STAGES) & 1u;
           if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kTimeoutNs)) {
@@ -378,7 +447,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // the leader's full barrier counts both CTAs' bytes
           const uint32_t fb = PAIR == 2 ? map_to_rank(full0 + 8 * s, 0) : full0 + 8 * s;
           const int kc = kb * BK;
-          if constexpr (PAIR == 1) {
+          if (FUSED && ph2) {
+            // down tile: h rows of the piece, four 64-column boxes of W_d
+            mbar_arrive_expect_tx(fb, G::STAGE_BYTES);
+            tma_load_2d(sa, &mapA2, fb, kc, arow);
+            const int c0 = tc.n * BN;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * B_BOX_BYTES, &mapB2, fb, c0 + 64 * j, kc, tc.e);
+          } else if constexpr (PAIR == 1) {
             mbar_arrive_expect_tx(fb, G::STAGE_BYTES);
             tma_load_2d(sa, &mapA, fb, kc, arow);
             if constexpr (MODE == MODE_GATE_UP_CONCAT) {
@@ -447,7 +523,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        const int nkb = (FUSED && t >= total1) ? p2.num_kb : p.num_kb;
+        for (int kb = 0; kb < nkb; ++kb) {
           const int s = it % G::STAGES;
           const uint32_t ph = static_cast<uint32_t>(it / G::STAGES) & 1u;
           if (!mbar_wait(full0 + 8 * s, ph, abort_flag, kTimeoutNs)) {
@@ -489,7 +566,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int part = (warp - 2) >> 2;  // which half of the tile's columns
     int ti = 0;
     for (int t = first_tile; t < total_tiles; t += tile_stride, ++ti) {
-      TileCoord tc = decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
+      const bool ph2 = FUSED && t >= total1;
+      TileCoord tc = ph2 ? decode_tile(t - total1, p2.n_tiles, p.E, s_mt, s_off, G::PIECE)
+                         : decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
       if constexpr (PAIR == 2) {
         tc.row0 += static_cast<int>(rank) * BM;
         tc.rows -= static_cast<int>(rank) * BM;  // may be <= 0: nothing of this half is stored
@@ -500,7 +579,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after_sync();
       const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
-      epilogue_tile<MODE>(p, tc, tacc, quad, part, lane, s_stage + (warp - 2) * kStageWarpBytes);
+      uint8_t* stage = s_stage + (warp - 2) * kStageWarpBytes;
+      if (ph2) {
+        epilogue_tile<MODE_DOWN>(p2, tc, tacc, quad, part, lane, stage);
+      } else {
+        epilogue_tile<MODE>(p, tc, tacc, quad, part, lane, stage);
+        if constexpr (FUSED) {
+          // publish this warp's h stores of the piece to the down tiles
+          fence_proxy_async_global();
+          __syncwarp();
+          if (lane == 0) red_release_add(arrivals + tc.piece, 1);
+        }
+      }
       tc_fence_before_sync();
       if constexpr (PAIR == 2) mbar_arrive_cluster(map_to_rank(tempty0 + 8 * acc, 0));
       else mbar_arrive(tempty0 + 8 * acc);
@@ -571,7 +661,7 @@ int max_pair_clusters(size_t smem, int num_sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<MODE, 2>, &cfg) != cudaSuccess || n <= 0)
+  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<MODE, 2, false>, &cfg) != cudaSuccess || n <= 0)
     n = num_sms / 2;
   cached = n;
   return n;
@@ -595,12 +685,13 @@ cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
   const int64_t max_pieces = p.R / Geo<PAIR>::PIECE + std::min(p.E, p.R);
   const int64_t max_tiles = max_pieces * p.n_tiles;
   const size_t smem = smem_bytes_for<PAIR>(p.E);
-  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, PAIR, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem_bytes_for<PAIR>(kMaxExperts)));
   if (err != cudaSuccess) return err;
   if constexpr (PAIR == 1) {
     const int grid = static_cast<int>(std::min<int64_t>(max_tiles, num_sms));
-    grouped_gemm_kernel<MODE, 1><<<grid, NUM_THREADS, smem, stream>>>(mapA, mapB, p);
+    grouped_gemm_kernel<MODE, 1, false><<<grid, NUM_THREADS, smem, stream>>>(mapA, mapB, mapA, mapB, p, p, nullptr);
     return cudaGetLastError();
   } else {
     const int clusters =
@@ -617,16 +708,16 @@ cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 2>, mapA, mapB, p);
+    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 2, false>, mapA, mapB, mapA, mapB, p, p,
+                              static_cast<int*>(nullptr));
   }
 }
 
+// Tensor maps and kernel parameters of one contraction.
 template <int MODE>
-cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t stream) {
-  if (a.R == 0) return cudaSuccess;
+cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& mapB, GemmParams& p) {
   const bool down = MODE == MODE_DOWN;
   const int K = down ? a.D : a.H;
-  CUtensorMap mapA, mapB;
   {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(a.R)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
@@ -650,7 +741,6 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t stream) {
     const cuuint32_t box[3] = {64, BK, 1};
     if (!encode_bf16_map(&mapB, a.W, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
-  GemmParams p;
   p.offsets = a.offsets;
   p.perm = a.perm;
   p.weights = a.weights;
@@ -667,8 +757,51 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t stream) {
   p.alpha = a.alpha;
   p.limit = a.limit;
   p.err_bit = down ? MOE_DEVICE_ERR_TIMEOUT_GEMM2 : MOE_DEVICE_ERR_TIMEOUT_GEMM1;
+  return cudaSuccess;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t stream) {
+  if (a.R == 0) return cudaSuccess;
+  CUtensorMap mapA, mapB;
+  GemmParams p;
+  cudaError_t err = prepare<MODE>(a, mapA, mapB, p);
+  if (err != cudaSuccess) return err;
   if (choose_pair(a.R, a.E) == 2) return launch_with<MODE, 2>(mapA, mapB, p, a.num_sms, stream);
   return launch_with<MODE, 1>(mapA, mapB, p, a.num_sms, stream);
+}
+
+template <int MODE>
+cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down, int* arrivals,
+                         cudaStream_t stream) {
+  if (up.R == 0) return cudaSuccess;
+  CUtensorMap mapA, mapB, mapA2, mapB2;
+  GemmParams p, p2;
+  cudaError_t err = prepare<MODE>(up, mapA, mapB, p);
+  if (err != cudaSuccess) return err;
+  err = prepare<MODE_DOWN>(down, mapA2, mapB2, p2);
+  if (err != cudaSuccess) return err;
+  // a timeout anywhere in the fused launch is reported as both stages'
+  p.err_bit = p2.err_bit = MOE_DEVICE_ERR_TIMEOUT_GEMM1 | MOE_DEVICE_ERR_TIMEOUT_GEMM2;
+  const int64_t max_pieces = p.R / BM + std::min(p.E, p.R);
+  const int64_t max_tiles = max_pieces * (p.n_tiles + p2.n_tiles);
+  const size_t smem = smem_bytes_for<1>(p.E);
+  err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, 1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_bytes_for<1>(kMaxExperts)));
+  if (err != cudaSuccess) return err;
+  // Cooperative: the launch fails rather than run with CTAs that are not
+  // resident, on which a down tile's wait could otherwise depend.
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(max_tiles, up.num_sms)));
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 1, true>, mapA, mapB, mapA2, mapB2, p, p2, arrivals);
 }
 
 }  // namespace
@@ -682,6 +815,14 @@ cudaError_t launch_gemm_gate_up(const GroupedGemmArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_gemm_down(const GroupedGemmArgs& a, cudaStream_t stream) {
   return launch_mode<MODE_DOWN>(a, stream);
+}
+
+int mega_ffn_counters(int R, int E) { return R / BM + std::min(E, R) + 1; }
+
+cudaError_t launch_mega_ffn(const GroupedGemmArgs& up, const GroupedGemmArgs& down, int* arrivals,
+                            cudaStream_t stream) {
+  return up.gate_up_format == 0 ? launch_fused<MODE_GATE_UP_CONCAT>(up, down, arrivals, stream)
+                                : launch_fused<MODE_GATE_UP_INTERLEAVED>(up, down, arrivals, stream);
 }
 
 }  // namespace moe

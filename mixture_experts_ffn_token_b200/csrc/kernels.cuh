@@ -47,9 +47,10 @@ cudaError_t launch_shared_index(int T, int Ns, int32_t* offsets, int32_t* perm, 
 
 // ----------------------------------------------------- gather and combine
 // scale (may be null): per-slot factor applied to the gathered row.
+// zero[0 .. n_zero) (may be null / 0) is cleared by the same launch.
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, const int32_t* offsets, int E, int R,
                           int k, int H, const float* scale, __nv_bfloat16* Xp, int* status, int num_sms,
-                          cudaStream_t stream);
+                          cudaStream_t stream, int* zero = nullptr, int n_zero = 0);
 // Ys (may be null, Ns = 0): shared-expert rows added after the routed ones;
 // mask (may be null): masked tokens get zero rows.
 cudaError_t launch_combine(const __nv_bfloat16* Y, int T, int H, int k, const __nv_bfloat16* Ys, int Ns,
@@ -77,6 +78,16 @@ struct GroupedGemmArgs {
 };
 cudaError_t launch_gemm_gate_up(const GroupedGemmArgs& a, cudaStream_t stream);
 cudaError_t launch_gemm_down(const GroupedGemmArgs& a, cudaStream_t stream);
+
+// Both contractions in one persistent cooperative launch: `up` describes the
+// gate_up GEMM (A = Xp, out = h) and `down` the down GEMM (A = h, out = Y,
+// which must not alias Xp).  A down tile of a 128-row piece waits (bounded)
+// until every gate_up tile of that piece has stored its h columns, counted
+// in arrivals[piece]; the counters must be zero at launch (launch_gather
+// clears them) and hold at least mega_ffn_counters(R, E) entries.
+int mega_ffn_counters(int R, int E);
+cudaError_t launch_mega_ffn(const GroupedGemmArgs& up, const GroupedGemmArgs& down, int* arrivals,
+                            cudaStream_t stream);
 
 // Resolves cuTensorMapEncodeTiled through the runtime (no libcuda link).
 bool tensor_map_encoder_available();

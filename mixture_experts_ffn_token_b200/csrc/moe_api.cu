@@ -1,6 +1,7 @@
 // moe_api.cu -- the C ABI declared in include/moe.h: host-side validation,
 // the workspace layout and the launch sequence of each entry point.
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -99,10 +100,17 @@ struct Extras {
 };
 
 struct WsLayout {
-  size_t status, chunk_counts, chunk_base, offsets, perm, idx, w, sink, xp, h, total;
-  // shared experts: CSR of the [T, Ns] slot space, Xp_s (then Y_s), h_s
-  size_t sh_offsets = 0, sh_perm = 0, sh_x = 0, sh_h = 0;
+  size_t status, chunk_counts, chunk_base, offsets, perm, idx, w, sink, xp, h, y, arr, total;
+  // shared experts: CSR of the [T, Ns] slot space, Xp_s, h_s, Y_s, counters
+  size_t sh_offsets = 0, sh_perm = 0, sh_x = 0, sh_h = 0, sh_y = 0, sh_arr = 0;
 };
+
+// Whether the two contractions run as one launch (the default) or as two;
+// MOE_B200_SINGLE_LAUNCH=0 selects two launches.
+bool single_launch() {
+  const char* env = std::getenv("MOE_B200_SINGLE_LAUNCH");
+  return !(env != nullptr && env[0] == '0');
+}
 
 WsLayout ws_layout(const moe_config_t* c, const Extras* ex = nullptr) {
   const size_t T = static_cast<size_t>(c->num_tokens), H = c->hidden_dim, E = c->num_experts, D = c->moe_dim;
@@ -130,6 +138,10 @@ WsLayout ws_layout(const moe_config_t* c, const Extras* ex = nullptr) {
   o += align256(R * H * 2);
   L.h = o;
   o += align256(R * D * 2);
+  L.y = o;  // Y [R, H] of the single-launch FFN (which still reads Xp while it writes Y)
+  o += align256(R * H * 2);
+  L.arr = o;
+  o += align256(static_cast<size_t>(moe::mega_ffn_counters(static_cast<int>(R), static_cast<int>(E))) * 4);
   if (ex != nullptr && ex->Ns > 0) {
     const size_t Rs = T * static_cast<size_t>(ex->Ns);
     L.sh_offsets = o;
@@ -140,6 +152,10 @@ WsLayout ws_layout(const moe_config_t* c, const Extras* ex = nullptr) {
     o += align256(Rs * H * 2);
     L.sh_h = o;
     o += align256(Rs * static_cast<size_t>(ex->Ds) * 2);
+    L.sh_y = o;
+    o += align256(Rs * H * 2);
+    L.sh_arr = o;
+    o += align256(static_cast<size_t>(moe::mega_ffn_counters(static_cast<int>(Rs), ex->Ns)) * 4);
   }
   L.total = o;
   return L;
@@ -197,18 +213,23 @@ struct Recorder {
 
 // One grouped expert FFN pass: gather (x rows by perm, times scale[slot] if
 // given) -> gate_up GEMM + activation -> down GEMM (+ bias, times
-// weights[slot] if given) writing Y at slot rows.  Y may alias xp (the
-// gate_up GEMM is done with it).  rec(base..base+2) before each kernel.
+// weights[slot] if given) writing Y at slot rows.  With two launches Y
+// overwrites Xp (the gate_up GEMM is done with it); the single launch
+// writes Y to y_sep and counts arrivals in arr.  *y_out = where Y is.
+// rec(base..base+2) before each stage (the down stage is empty when fused).
 moe_status_t enqueue_grouped_pass(const moe_config_t* c, int E, int k, int D, const void* x, const void* gate_up_w,
                                   const void* gate_up_b, const void* down_w, const void* down_b,
                                   const int32_t* offsets, const int32_t* perm, const float* scale,
-                                  const float* weights, __nv_bfloat16* xp, __nv_bfloat16* h, __nv_bfloat16* y,
-                                  int* status, int num_sms, cudaStream_t stream, const Recorder& rec, int base) {
+                                  const float* weights, __nv_bfloat16* xp, __nv_bfloat16* h, __nv_bfloat16* y_sep,
+                                  int* arr, __nv_bfloat16** y_out, int* status, int num_sms, cudaStream_t stream,
+                                  const Recorder& rec, int base) {
   const int T = c->num_tokens, H = c->hidden_dim;
   const int R = T * k;
+  const bool fused = single_launch();
   rec(base);
   if (moe::launch_gather(static_cast<const __nv_bfloat16*>(x), perm, offsets, E, R, k, H, scale, xp, status,
-                         num_sms, stream) != cudaSuccess)
+                         num_sms, stream, fused ? arr : nullptr, fused ? moe::mega_ffn_counters(R, E) : 0) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
   moe::GroupedGemmArgs g;
   g.offsets = offsets;
@@ -230,14 +251,21 @@ moe_status_t enqueue_grouped_pass(const moe_config_t* c, int E, int k, int D, co
   g.W = static_cast<const __nv_bfloat16*>(gate_up_w);
   g.bias = static_cast<const __nv_bfloat16*>(gate_up_b);
   g.out = h;
+  moe::GroupedGemmArgs g2 = g;
+  g2.A = h;
+  g2.W = static_cast<const __nv_bfloat16*>(down_w);
+  g2.bias = static_cast<const __nv_bfloat16*>(down_b);
+  g2.out = fused ? y_sep : xp;
+  *y_out = g2.out;
   rec(base + 1);
+  if (fused) {
+    if (moe::launch_mega_ffn(g, g2, arr, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    rec(base + 2);
+    return MOE_OK;
+  }
   if (moe::launch_gemm_gate_up(g, stream) != cudaSuccess) return MOE_ERR_CUDA;
-  g.A = h;
-  g.W = static_cast<const __nv_bfloat16*>(down_w);
-  g.bias = static_cast<const __nv_bfloat16*>(down_b);
-  g.out = y;
   rec(base + 2);
-  if (moe::launch_gemm_down(g, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_gemm_down(g2, stream) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
@@ -250,12 +278,14 @@ moe_status_t enqueue_ffn(const moe_config_t* c, const void* x, const void* gate_
                          cudaStream_t stream, cudaEvent_t const* ev) {
   const Recorder rec{ev, stream};
   __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
+  __nv_bfloat16* y = nullptr;
   moe_status_t st = enqueue_grouped_pass(c, c->num_experts, c->top_k, c->moe_dim, x, gate_up_w, gate_up_b, down_w,
                                          down_b, offsets, perm, nullptr, weights, xp, at<__nv_bfloat16>(ws, L.h),
-                                         xp, at<int>(ws, L.status), num_sms, stream, rec, 0);
+                                         at<__nv_bfloat16>(ws, L.y), at<int>(ws, L.arr), &y, at<int>(ws, L.status),
+                                         num_sms, stream, rec, 0);
   if (st != MOE_OK) return st;
   rec(3);
-  if (moe::launch_combine(xp, c->num_tokens, c->hidden_dim, c->top_k, nullptr, 0, nullptr,
+  if (moe::launch_combine(y, c->num_tokens, c->hidden_dim, c->top_k, nullptr, 0, nullptr,
                           static_cast<__nv_bfloat16*>(out), num_sms, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   rec(4);
@@ -364,9 +394,11 @@ moe_status_t forward_impl(const moe_config_t* cfg, const moe_extras_t* extras, c
 
   // routed pass: the weight scales the input (weight first) or the output
   __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
+  __nv_bfloat16* y = nullptr;
   st = enqueue_grouped_pass(cfg, cfg->num_experts, k, cfg->moe_dim, x, gate_up_w, gate_up_b, down_w, down_b, offsets,
                             perm, ex.weight_first ? w : nullptr, ex.weight_first ? nullptr : w, xp,
-                            at<__nv_bfloat16>(ws, L.h), xp, status, num_sms, stream, rec, 4);
+                            at<__nv_bfloat16>(ws, L.h), at<__nv_bfloat16>(ws, L.y), at<int>(ws, L.arr), &y, status,
+                            num_sms, stream, rec, 4);
   if (st != MOE_OK) return st;
   __nv_bfloat16* ys = nullptr;
   rec(7);
@@ -377,16 +409,17 @@ moe_status_t forward_impl(const moe_config_t* cfg, const moe_extras_t* extras, c
     int32_t* s_perm = at<int32_t>(ws, L.sh_perm);
     if (moe::launch_shared_index(T, ex.Ns, s_off, s_perm, num_sms, stream) != cudaSuccess) return MOE_ERR_CUDA;
     const float* gates = cfg->router == MOE_ROUTER_SIGMOID_SINK ? sink : nullptr;
-    ys = at<__nv_bfloat16>(ws, L.sh_x);
     st = enqueue_grouped_pass(cfg, ex.Ns, ex.Ns, ex.Ds, x, ex.s_gu_w, ex.s_gu_b, ex.s_d_w, ex.s_d_b, s_off, s_perm,
-                              ex.weight_first ? gates : nullptr, ex.weight_first ? nullptr : gates, ys,
-                              at<__nv_bfloat16>(ws, L.sh_h), ys, status, num_sms, stream, rec, 8);
+                              ex.weight_first ? gates : nullptr, ex.weight_first ? nullptr : gates,
+                              at<__nv_bfloat16>(ws, L.sh_x), at<__nv_bfloat16>(ws, L.sh_h),
+                              at<__nv_bfloat16>(ws, L.sh_y), at<int>(ws, L.sh_arr), &ys, status, num_sms, stream,
+                              rec, 8);
     if (st != MOE_OK) return st;
   } else {
     for (int i = 8; i <= 10; ++i) rec(i);
   }
   rec(11);
-  if (moe::launch_combine(xp, T, cfg->hidden_dim, k, ys, ex.Ns, ex.mask, static_cast<__nv_bfloat16*>(out), num_sms,
+  if (moe::launch_combine(y, T, cfg->hidden_dim, k, ys, ex.Ns, ex.mask, static_cast<__nv_bfloat16*>(out), num_sms,
                           stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   rec(12);
@@ -407,6 +440,12 @@ const char* moe_status_string(moe_status_t status) {
     case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
   }
   return "MOE_ERR_UNKNOWN";
+}
+
+moe_status_t moe_single_launch_ffn(int32_t* enabled) {
+  if (enabled == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  *enabled = single_launch() ? 1 : 0;
+  return MOE_OK;
 }
 
 moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {

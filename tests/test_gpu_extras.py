@@ -38,7 +38,9 @@ def test_shared_experts(wl):
     run_and_check_ex(wl, seed=3)
 
 
-def test_everything_together():
+@pytest.mark.parametrize("single_launch", ["1", "0"])
+def test_everything_together(single_launch, monkeypatch):
+    monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", single_launch)
     run_and_check_ex(SNK.replace(num_shared=2, shared_dim=136, weight_first=True, mask_frac=0.25), seed=4)
     run_and_check_ex(GPT.replace(num_shared=1, shared_dim=200, weight_first=True, mask_frac=0.5), seed=5)
 

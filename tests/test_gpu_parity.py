@@ -35,21 +35,48 @@ def test_forward_small(name):
     run_and_check(SMALL[name], seed=0)
 
 
-@pytest.mark.parametrize("pair", ["1", "2"])
+# GEMM variants: both contractions in one cooperative launch (default), two
+# launches of one CTA per 128x256 tile, or two launches of a CTA pair per
+# 256x256 tile (tcgen05 cta_group::2).
+VARIANTS = {"single_launch": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1"},
+            "two_launches": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "1"},
+            "two_launches_cta_pair": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "2"}}
+
+
+def set_variant(monkeypatch, variant):
+    for k, v in VARIANTS[variant].items():
+        monkeypatch.setenv(k, v)
+
+
+@pytest.mark.parametrize("variant", sorted(VARIANTS))
 @pytest.mark.parametrize("name", sorted(SMALL))
-def test_forward_small_each_cta_variant(name, pair, monkeypatch):
-    """Both GEMM variants on every layout: one CTA per 128x256 tile, or a CTA
-    pair on a 256x256 tile (tcgen05 cta_group::2)."""
-    monkeypatch.setenv("MOE_B200_CTA_PAIR", pair)
+def test_forward_small_each_gemm_variant(name, variant, monkeypatch):
+    set_variant(monkeypatch, variant)
+    assert abi.moe_single_launch_ffn() == (variant == "single_launch")
     run_and_check(SMALL[name], seed=1)
 
 
-@pytest.mark.parametrize("pair", ["1", "2"])
-def test_forward_mixtral_shape_each_cta_variant(pair, monkeypatch):
-    monkeypatch.setenv("MOE_B200_CTA_PAIR", pair)
+@pytest.mark.parametrize("variant", sorted(VARIANTS))
+def test_forward_mixtral_shape_each_gemm_variant(variant, monkeypatch):
+    set_variant(monkeypatch, variant)
     wl = WORKLOADS["mixtral"].replace(num_tokens=1024, hidden_dim=1024, moe_dim=1536,
                                       logits_std=0.02 * math.sqrt(1024))
     run_and_check(wl, seed=2)
+
+
+@pytest.mark.parametrize("name", sorted(SMALL) + ["many_pieces"])
+def test_single_launch_equals_two_launches(name, monkeypatch):
+    """The single launch does the same tiles, MMAs and epilogues as the two
+    launches, only scheduled differently: the outputs are identical bit for bit."""
+    wl = SMALL.get(name) or WORKLOADS["sink"].replace(num_tokens=2000, hidden_dim=512, moe_dim=256)
+    d = to_dev(make_inputs(wl, 11))
+    outs = []
+    for mode in ("1", "0"):
+        monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", mode)
+        run = GpuRun(wl, d)
+        assert run.status == 0
+        outs.append(run.out.clone())
+    assert torch.equal(outs[0], outs[1])
 
 
 @pytest.mark.parametrize("seed", [1, 2])
