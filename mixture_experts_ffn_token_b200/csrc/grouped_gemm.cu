@@ -88,6 +88,7 @@ struct GemmParams {
   int activation;
   float alpha, limit;
   int err_bit;
+  int b_one_box;  // 1: the B tensor map delivers a stage's whole B tile in one copy
 };
 
 struct TileCoord {
@@ -448,12 +449,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t fb = PAIR == 2 ? map_to_rank(full0 + 8 * s, 0) : full0 + 8 * s;
           const int kc = kb * BK;
           if (FUSED && ph2) {
-            // down tile: h rows of the piece, four 64-column boxes of W_d
+            // down tile: h rows of the piece, 256 columns of W_d
             mbar_arrive_expect_tx(fb, G::STAGE_BYTES);
             tma_load_2d(sa, &mapA2, fb, kc, arow);
-            const int c0 = tc.n * BN;
+            if (p2.b_one_box) {
+              tma_load_4d(sb, &mapB2, fb, 0, kc, 4 * tc.n, tc.e);
+            } else {
+              const int c0 = tc.n * BN;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * B_BOX_BYTES, &mapB2, fb, c0 + 64 * j, kc, tc.e);
+              for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * B_BOX_BYTES, &mapB2, fb, c0 + 64 * j, kc, tc.e);
+            }
+          } else if (PAIR == 1 && p.b_one_box) {
+            // {64 columns, K, column block, (gate/up,) E} view: one copy lays
+            // the four 64-column boxes out exactly as four copies would
+            mbar_arrive_expect_tx(fb, G::STAGE_BYTES);
+            tma_load_2d(sa, &mapA, fb, kc, arow);
+            if constexpr (MODE == MODE_GATE_UP_CONCAT) tma_load_5d(sb, &mapB, fb, 0, kc, 2 * tc.n, 0, tc.e);
+            else tma_load_4d(sb, &mapB, fb, 0, kc, 4 * tc.n, tc.e);
           } else if constexpr (PAIR == 1) {
             mbar_arrive_expect_tx(fb, G::STAGE_BYTES);
             tma_load_2d(sa, &mapA, fb, kc, arow);
@@ -672,6 +684,13 @@ int max_pair_clusters(size_t smem, int num_sms) {
 // part's power limit, where it draws more power, runs at a lower clock and
 // ends no faster; the single-CTA kernel is therefore the default.
 // MOE_B200_CTA_PAIR=2 selects the pair variant (1 forces the default).
+// One-copy B loads (default) or four 64-column copies per stage
+// (MOE_B200_B_ONE_BOX=0).
+bool one_box_enabled() {
+  const char* env = std::getenv("MOE_B200_B_ONE_BOX");
+  return !(env != nullptr && env[0] == '0');
+}
+
 int choose_pair(int /*R*/, int /*E*/) {
   if (const char* env = std::getenv("MOE_B200_CTA_PAIR")) {
     if (env[0] == '2') return 2;
@@ -714,8 +733,40 @@ cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
 }
 
 // Tensor maps and kernel parameters of one contraction.
+// B tensor map that delivers a whole 64 K x 256 column stage tile in one copy:
+// {64 columns, K, column blocks (, gate/up), E}, the column-block dimension
+// 128 bytes apart, box {64, 64, blocks (, 2), 1}.  Its shared-memory image
+// equals that of the four 64-column boxes of the plain view (the swizzle
+// depends only on the shared address).  Requires the columns of one half to
+// be a multiple of 64, so that every in-range coordinate stays inside the
+// tensor; otherwise (or if the driver declines the view) false.
 template <int MODE>
-cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& mapB, GemmParams& p) {
+bool encode_one_box_b(const GroupedGemmArgs& a, CUtensorMap* map) {
+  const cuuint64_t H = a.H, D = a.D, E = a.E;
+  if (MODE == MODE_GATE_UP_CONCAT) {
+    if (D % 64 != 0) return false;
+    const cuuint64_t dims[5] = {64, H, D / 64, 2, E};
+    const cuuint64_t strides[4] = {2 * D * 2, 128, D * 2, H * 2 * D * 2};
+    const cuuint32_t box[5] = {64, BK, 2, 2, 1};
+    return encode_bf16_map(map, a.W, 5, dims, strides, box);
+  } else if (MODE == MODE_GATE_UP_INTERLEAVED) {
+    if ((2 * D) % 64 != 0) return false;
+    const cuuint64_t dims[4] = {64, H, 2 * D / 64, E};
+    const cuuint64_t strides[3] = {2 * D * 2, 128, H * 2 * D * 2};
+    const cuuint32_t box[4] = {64, BK, 4, 1};
+    return encode_bf16_map(map, a.W, 4, dims, strides, box);
+  } else {
+    if (H % 64 != 0) return false;
+    const cuuint64_t dims[4] = {64, D, H / 64, E};
+    const cuuint64_t strides[3] = {H * 2, 128, D * H * 2};
+    const cuuint32_t box[4] = {64, BK, 4, 1};
+    return encode_bf16_map(map, a.W, 4, dims, strides, box);
+  }
+}
+
+template <int MODE>
+cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& mapB, GemmParams& p,
+                    bool allow_one_box) {
   const bool down = MODE == MODE_DOWN;
   const int K = down ? a.D : a.H;
   {
@@ -725,7 +776,10 @@ cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& ma
     if (!encode_bf16_map(&mapA, a.A, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
   const cuuint64_t H = a.H, D = a.D, E = a.E;
-  if (MODE == MODE_GATE_UP_CONCAT) {
+  p.b_one_box = allow_one_box && one_box_enabled() && encode_one_box_b<MODE>(a, &mapB) ? 1 : 0;
+  if (p.b_one_box) {
+    // mapB already holds the one-copy view
+  } else if (MODE == MODE_GATE_UP_CONCAT) {
     const cuuint64_t dims[4] = {D, 2, H, E};
     const cuuint64_t strides[3] = {D * 2, 2 * D * 2, H * 2 * D * 2};
     const cuuint32_t box[4] = {64, 1, BK, 1};
@@ -765,9 +819,10 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t stream) {
   if (a.R == 0) return cudaSuccess;
   CUtensorMap mapA, mapB;
   GemmParams p;
-  cudaError_t err = prepare<MODE>(a, mapA, mapB, p);
+  const int pair = choose_pair(a.R, a.E);
+  cudaError_t err = prepare<MODE>(a, mapA, mapB, p, pair == 1);
   if (err != cudaSuccess) return err;
-  if (choose_pair(a.R, a.E) == 2) return launch_with<MODE, 2>(mapA, mapB, p, a.num_sms, stream);
+  if (pair == 2) return launch_with<MODE, 2>(mapA, mapB, p, a.num_sms, stream);
   return launch_with<MODE, 1>(mapA, mapB, p, a.num_sms, stream);
 }
 
@@ -777,9 +832,9 @@ cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down,
   if (up.R == 0) return cudaSuccess;
   CUtensorMap mapA, mapB, mapA2, mapB2;
   GemmParams p, p2;
-  cudaError_t err = prepare<MODE>(up, mapA, mapB, p);
+  cudaError_t err = prepare<MODE>(up, mapA, mapB, p, true);
   if (err != cudaSuccess) return err;
-  err = prepare<MODE_DOWN>(down, mapA2, mapB2, p2);
+  err = prepare<MODE_DOWN>(down, mapA2, mapB2, p2, true);
   if (err != cudaSuccess) return err;
   // a timeout anywhere in the fused launch is reported as both stages'
   p.err_bit = p2.err_bit = MOE_DEVICE_ERR_TIMEOUT_GEMM1 | MOE_DEVICE_ERR_TIMEOUT_GEMM2;

@@ -37,9 +37,12 @@ def test_forward_small(name):
 
 # GEMM variants: both contractions in one cooperative launch (default), two
 # launches of one CTA per 128x256 tile, or two launches of a CTA pair per
-# 256x256 tile (tcgen05 cta_group::2).
-VARIANTS = {"single_launch": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1"},
-            "two_launches": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "1"},
+# 256x256 tile (tcgen05 cta_group::2); B stage tiles in one copy (default
+# where the column count allows) or in four 64-column copies.
+VARIANTS = {"single_launch": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1", "MOE_B200_B_ONE_BOX": "1"},
+            "single_launch_four_box": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1",
+                                       "MOE_B200_B_ONE_BOX": "0"},
+            "two_launches": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "1", "MOE_B200_B_ONE_BOX": "1"},
             "two_launches_cta_pair": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "2"}}
 
 
@@ -52,7 +55,7 @@ def set_variant(monkeypatch, variant):
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_forward_small_each_gemm_variant(name, variant, monkeypatch):
     set_variant(monkeypatch, variant)
-    assert abi.moe_single_launch_ffn() == (variant == "single_launch")
+    assert abi.moe_single_launch_ffn() == variant.startswith("single_launch")
     run_and_check(SMALL[name], seed=1)
 
 
@@ -64,19 +67,37 @@ def test_forward_mixtral_shape_each_gemm_variant(variant, monkeypatch):
     run_and_check(wl, seed=2)
 
 
-@pytest.mark.parametrize("name", sorted(SMALL) + ["many_pieces"])
+# column counts that are multiples of 64 (one-copy B tiles) in every layout
+ALIGNED = {
+    "concat_silu": WORKLOADS["sink"].replace(num_tokens=2000, hidden_dim=512, moe_dim=256),
+    "interleaved_bias": WORKLOADS["gptoss"].replace(num_tokens=160, hidden_dim=384, num_experts=16, moe_dim=160),
+    "concat_gelu_ragged_k": WORKLOADS["decode"].replace(num_tokens=24, hidden_dim=328, num_experts=16, moe_dim=192),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL) + sorted(ALIGNED))
 def test_single_launch_equals_two_launches(name, monkeypatch):
     """The single launch does the same tiles, MMAs and epilogues as the two
-    launches, only scheduled differently: the outputs are identical bit for bit."""
-    wl = SMALL.get(name) or WORKLOADS["sink"].replace(num_tokens=2000, hidden_dim=512, moe_dim=256)
+    launches, only scheduled differently; a one-copy B stage tile has the same
+    shared-memory image as four 64-column copies: every variant's output is
+    identical bit for bit."""
+    wl = SMALL.get(name) or ALIGNED[name]
     d = to_dev(make_inputs(wl, 11))
     outs = []
-    for mode in ("1", "0"):
-        monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", mode)
+    for single, one_box in (("1", "1"), ("0", "1"), ("1", "0"), ("0", "0")):
+        monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", single)
+        monkeypatch.setenv("MOE_B200_B_ONE_BOX", one_box)
         run = GpuRun(wl, d)
         assert run.status == 0
         outs.append(run.out.clone())
-    assert torch.equal(outs[0], outs[1])
+    for o in outs[1:]:
+        assert torch.equal(outs[0], o)
+
+
+@pytest.mark.parametrize("name", sorted(ALIGNED))
+def test_one_box_layouts_against_oracle(name, monkeypatch):
+    monkeypatch.setenv("MOE_B200_B_ONE_BOX", "1")
+    run_and_check(ALIGNED[name], seed=12)
 
 
 @pytest.mark.parametrize("seed", [1, 2])
