@@ -145,6 +145,9 @@ __global__ void __launch_bounds__(kCsrThreads) csr_scatter_kernel(const int32_t*
   }
 }
 
+constexpr int kCombineBatch = 8;   // rows a combine thread loads before summing
+constexpr int kGatherUnroll = 4;   // 16-byte chunks a gather lane loads before storing
+
 // One warp per gathered row: Xp[p, :] = x[perm[p] / k, :] (times
 // scale[perm[p]] when scale is given), 16-byte vectors.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ x,
@@ -172,19 +175,26 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
     }
     const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(s / k) * H);
     uint4* dst = reinterpret_cast<uint4*>(Xp + p * H);
-    if (scale == nullptr) {
-      for (int c = lane; c < vec; c += 32) dst[c] = __ldg(src + c);
-    } else {
-      // apply_router_weight_first: the routing weight scales the expert input
-      const float f = scale[s];
-      for (int c = lane; c < vec; c += 32) {
-        const uint4 v = __ldg(src + c);
-        uint4 o;
-        o.x = pack_bf16x2(bf16_lo(v.x) * f, bf16_hi(v.x) * f);
-        o.y = pack_bf16x2(bf16_lo(v.y) * f, bf16_hi(v.y) * f);
-        o.z = pack_bf16x2(bf16_lo(v.z) * f, bf16_hi(v.z) * f);
-        o.w = pack_bf16x2(bf16_lo(v.w) * f, bf16_hi(v.w) * f);
-        dst[c] = o;
+    // apply_router_weight_first: the routing weight scales the expert input
+    const float f = scale != nullptr ? scale[s] : 1.f;
+    // kGatherUnroll chunks per lane in flight before their stores
+    for (int c0 = lane; c0 < vec; c0 += 32 * kGatherUnroll) {
+      uint4 v[kGatherUnroll];
+#pragma unroll
+      for (int q = 0; q < kGatherUnroll; ++q)
+        if (c0 + 32 * q < vec) v[q] = __ldg(src + c0 + 32 * q);
+#pragma unroll
+      for (int q = 0; q < kGatherUnroll; ++q) {
+        if (c0 + 32 * q < vec) {
+          uint4 o = v[q];
+          if (scale != nullptr) {
+            o.x = pack_bf16x2(bf16_lo(o.x) * f, bf16_hi(o.x) * f);
+            o.y = pack_bf16x2(bf16_lo(o.y) * f, bf16_hi(o.y) * f);
+            o.z = pack_bf16x2(bf16_lo(o.z) * f, bf16_hi(o.z) * f);
+            o.w = pack_bf16x2(bf16_lo(o.w) * f, bf16_hi(o.w) * f);
+          }
+          dst[c0 + 32 * q] = o;
+        }
       }
     }
   }
@@ -205,14 +215,29 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
     const int c = static_cast<int>(i - t * vec);
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (mask == nullptr || mask[t] != 0) {
-      for (int j = 0; j < k + Ns; ++j) {
-        const __nv_bfloat16* row = j < k ? Y + (t * k + j) * H : Ys + (t * Ns + (j - k)) * H;
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(row) + c);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      const int terms = k + Ns;
+      // up to kCombineBatch rows in flight per thread: all loads of a batch
+      // are issued before the first add (the sum order stays j ascending)
+      for (int j0 = 0; j0 < terms; j0 += kCombineBatch) {
+        uint4 v[kCombineBatch];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          acc[2 * q] += bf16_lo(w[q]);
-          acc[2 * q + 1] += bf16_hi(w[q]);
+        for (int q = 0; q < kCombineBatch; ++q) {
+          const int j = j0 + q;
+          if (j < terms) {
+            const __nv_bfloat16* row = j < k ? Y + (t * k + j) * H : Ys + (t * Ns + (j - k)) * H;
+            v[q] = __ldg(reinterpret_cast<const uint4*>(row) + c);
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < kCombineBatch; ++q) {
+          if (j0 + q < terms) {
+            const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              acc[2 * r] += bf16_lo(w[r]);
+              acc[2 * r + 1] += bf16_hi(w[r]);
+            }
+          }
         }
       }
     }

@@ -72,6 +72,14 @@ struct Geo {
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM * PAIR, BN, /*a_mn_major=*/false, /*b_mn_major=*/true);
 };
 
+// Half tiles (single-CTA tiles only): an expert's last row piece with at most
+// 64 valid rows is multiplied with M = 64 MMAs, half the tensor work of the
+// full 128-row tile.  The M = 64 accumulator of tcgen05 (cta_group::1) puts
+// row r in TMEM lane 32*(r/16) + r%16: the first 16 lanes of each 32-lane
+// quadrant, so epilogue warp q reads rows 16q .. 16q+15 from its own lanes.
+constexpr int HALF_ROWS = 64;
+constexpr uint32_t IDESC_HALF = idesc_bf16_f32(HALF_ROWS, BN, /*a_mn_major=*/false, /*b_mn_major=*/true);
+
 constexpr int MODE_GATE_UP_CONCAT = 0;
 constexpr int MODE_GATE_UP_INTERLEAVED = 1;
 constexpr int MODE_DOWN = 2;
@@ -245,13 +253,15 @@ __device__ __forceinline__ void down_chunk(const GemmParams& p, const TileCoord&
 // One tile's epilogue for one warp: rows quad*32.., output columns of `part`.
 template <int MODE>
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int quad,
-                                              int part, int lane, uint8_t* stage) {
+                                              int part, int lane, uint8_t* stage, bool half) {
   constexpr bool kDown = MODE == MODE_DOWN;
-  const int row = quad * 32 + lane;
+  // tile row held by this thread's TMEM lane (half tiles: lanes 0..15 of the quadrant)
+  const int row = half ? quad * 16 + lane : quad * 32 + lane;
+  const bool has_row = !half || lane < 16;
   // destination row of this thread's tile row, or -1 if it is not stored
   int64_t dst = -1;
   float wgt = 0.f;
-  if (row < tc.rows) {
+  if (has_row && row < tc.rows) {
     if constexpr (kDown) {
       const int slot = p.perm[tc.row0 + row];
       if (slot < 0 || slot >= p.R) {
@@ -535,7 +545,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        const int nkb = (FUSED && t >= total1) ? p2.num_kb : p.num_kb;
+        const bool ph2 = FUSED && t >= total1;
+        const int nkb = ph2 ? p2.num_kb : p.num_kb;
+        uint32_t idesc = G::IDESC;
+        if constexpr (PAIR == 1) {
+          const TileCoord tc = ph2 ? decode_tile(t - total1, p2.n_tiles, p.E, s_mt, s_off, G::PIECE)
+                                   : decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
+          if (tc.rows <= HALF_ROWS) idesc = IDESC_HALF;
+        }
         for (int kb = 0; kb < nkb; ++kb) {
           const int s = it % G::STAGES;
           const uint32_t ph = static_cast<uint32_t>(it / G::STAGES) & 1u;
@@ -555,7 +572,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // groups 1024 B apart (SBO); a 16-row K step is 2048 B.
             const uint64_t b_desc = smem_desc_sw128(sb + kk * UMMA_K * 128, B_BOX_BYTES, 1024);
             if constexpr (PAIR == 2) mma_bf16_ss_pair(d_tmem, a_desc, b_desc, G::IDESC, (kb | kk) != 0 ? 1u : 0u);
-            else mma_bf16_ss(d_tmem, a_desc, b_desc, G::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            else mma_bf16_ss(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           if constexpr (PAIR == 2) mma_commit_pair(empty0 + 8 * s, 0x3);
           else mma_commit(empty0 + 8 * s);
@@ -592,10 +609,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after_sync();
       const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
       uint8_t* stage = s_stage + (warp - 2) * kStageWarpBytes;
+      const bool half = PAIR == 1 && tc.rows <= HALF_ROWS;
       if (ph2) {
-        epilogue_tile<MODE_DOWN>(p2, tc, tacc, quad, part, lane, stage);
+        epilogue_tile<MODE_DOWN>(p2, tc, tacc, quad, part, lane, stage, half);
       } else {
-        epilogue_tile<MODE>(p, tc, tacc, quad, part, lane, stage);
+        epilogue_tile<MODE>(p, tc, tacc, quad, part, lane, stage, half);
         if constexpr (FUSED) {
           // publish this warp's h stores of the piece to the down tiles
           fence_proxy_async_global();
