@@ -150,6 +150,30 @@ __device__ __forceinline__ int ld_acquire(const int* addr) {
   return v;
 }
 
+// Dynamic tile order of the single launch (when `sched` is given): the producer thread draws tile
+// numbers from a global counter (one tile ahead, so the atomic's latency
+// overlaps the current tile's copies) and hands each to the MMA thread and
+// the epilogue warps through a ring of kTileRing slots in shared memory.
+// Numbers are drawn in increasing order, so a down tile still only waits on
+// tiles that were handed to running CTAs before it; CTAs that finish early
+// simply draw more tiles, which evens out the end of the launch.  Without
+// `sched` CTA c takes tiles c, c + grid, c + 2 grid, ... (static order).
+constexpr int kTileRing = 8;
+
+// Consumer side of the ring: the n-th tile number (n counts from 0), or
+// false if the wait gave up.  Every lane of the calling warp reads the slot
+// before `releaser` frees it.
+__device__ __forceinline__ bool ring_take(uint32_t ring_full0, uint32_t ring_empty0, const volatile int* ring,
+                                          int n, volatile int* abort, bool releaser, int* t) {
+  const int slot = n % kTileRing;
+  const uint32_t ph = static_cast<uint32_t>(n / kTileRing) & 1u;
+  if (!mbar_wait(ring_full0 + 8 * slot, ph, abort, kTimeoutNs)) return false;
+  *t = ring[slot];
+  __syncwarp(__activemask());
+  if (releaser) mbar_arrive(ring_empty0 + 8 * slot);
+  return true;
+}
+
 // Bounded wait for *counter >= target.  Gives up (false, CTA abort raised,
 // err bits recorded at once so other CTAs stop waiting too) after the
 // timeout, when this CTA aborts, or when another CTA has recorded a timeout.
@@ -323,7 +347,7 @@ template <int MODE, int PAIR, bool FUSED>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                         const __grid_constant__ CUtensorMap mapA2, const __grid_constant__ CUtensorMap mapB2,
-                        const GemmParams p, const GemmParams p2, int* arrivals) {
+                        const GemmParams p, const GemmParams p2, int* arrivals, int* sched) {
   static_assert(!FUSED || (PAIR == 1 && MODE != MODE_DOWN), "the fused form is gate_up then down, one CTA a tile");
   using G = Geo<PAIR>;
   extern __shared__ uint8_t smem_raw[];
@@ -335,10 +359,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tfull0 = empty0 + 8 * G::STAGES;     // 2 mbarriers
   const uint32_t tempty0 = tfull0 + 16;               // 2 mbarriers
   const uint32_t drain_bar = tempty0 + 16;            // 1 mbarrier
-  static_assert((2 * G::STAGES + 5) * 8 <= 256, "mbarriers overflow their part of the control block");
+  const uint32_t ring_full0 = drain_bar + 8;          // kTileRing mbarriers (FUSED)
+  const uint32_t ring_empty0 = ring_full0 + 8 * kTileRing;  // kTileRing mbarriers (FUSED)
+  static_assert((2 * G::STAGES + 5 + (FUSED ? 2 * kTileRing : 0)) * 8 <= 256,
+                "mbarriers overflow their part of the control block");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 256);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 260);
   int* bad_flag = reinterpret_cast<int*>(ctrl + 264);
+  volatile int* s_ring = reinterpret_cast<volatile int*>(ctrl + 288);  // kTileRing tile numbers
   int* s_off = reinterpret_cast<int*>(ctrl + CTRL_BYTES);
   int* s_mt = s_off + (p.E + 1);
   // epilogue staging: one kStageWarpBytes block per epilogue warp, 16-byte aligned
@@ -360,6 +388,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(tempty0 + 8 * a, 32 * NUM_EPI_WARPS * PAIR);
     }
     mbar_init(drain_bar, 1);
+    if constexpr (FUSED) {
+      for (int i = 0; i < kTileRing; ++i) {
+        mbar_init(ring_full0 + 8 * i, 1);
+        mbar_init(ring_empty0 + 8 * i, 1 + NUM_EPI_WARPS);  // the MMA thread and one lane per epilogue warp
+      }
+    }
     *abort_flag = 0;
     *bad_flag = 0;
     fence_mbar_init();
@@ -425,13 +459,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // down tiles of a piece wait for this many arrivals (one per epilogue warp
   // of each of the piece's gate_up tiles)
   const int arrivals_needed = NUM_EPI_WARPS * p.n_tiles;
+  const bool dyn = FUSED && sched != nullptr;  // dynamic tile order
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
       int it = 0;
       bool ok = true;
-      for (int t = first_tile; ok && t < total_tiles; t += tile_stride) {
+      int t_next = dyn ? atomicAdd(sched, 1) : first_tile;
+      for (int n = 0; ok; ++n) {
+        const int t = t_next;
+        if (dyn) {
+          // hand tile number n to the consumers (the end marker too)
+          const int slot = n % kTileRing;
+          if (!mbar_wait(ring_empty0 + 8 * slot, (static_cast<uint32_t>(n / kTileRing) & 1u) ^ 1u, abort_flag,
+                         kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          s_ring[slot] = t;
+          mbar_arrive(ring_full0 + 8 * slot);
+          if (t >= total_tiles) break;
+          t_next = atomicAdd(sched, 1);  // in flight while this tile's copies are issued
+        } else {
+          if (t >= total_tiles) break;
+          t_next = t + tile_stride;
+        }
         const bool ph2 = FUSED && t >= total1;
         const TileCoord tc = ph2 ? decode_tile(t - total1, p2.n_tiles, p.E, s_mt, s_off, G::PIECE)
                                  : decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
@@ -534,9 +587,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // --------------------------------------------------- MMA issuer
-      int it = 0, ti = 0;
+      int it = 0;
       bool ok = true;
-      for (int t = first_tile; ok && t < total_tiles; t += tile_stride, ++ti) {
+      for (int ti = 0; ok; ++ti) {
+        int t = first_tile + ti * tile_stride;
+        if (dyn) {
+          if (!ring_take(ring_full0, ring_empty0, s_ring, ti, abort_flag, true, &t)) {
+            ok = false;
+            break;
+          }
+        }
+        if (t >= total_tiles) break;
         const int acc = ti & 1;
         const uint32_t aph = static_cast<uint32_t>(ti >> 1) & 1u;
         if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, abort_flag, kTimeoutNs)) {
@@ -593,8 +654,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------ epilogue
     const int quad = warp & 3;  // this warp may access TMEM lanes 32*quad..+31
     const int part = (warp - 2) >> 2;  // which half of the tile's columns
-    int ti = 0;
-    for (int t = first_tile; t < total_tiles; t += tile_stride, ++ti) {
+    for (int ti = 0;; ++ti) {
+      int t = first_tile + ti * tile_stride;
+      if (dyn) {
+        const bool took = ring_take(ring_full0, ring_empty0, s_ring, ti, abort_flag, lane == 0, &t);
+        if (!__all_sync(0xffffffffu, took)) break;
+      }
+      if (t >= total_tiles) break;
       const bool ph2 = FUSED && t >= total1;
       TileCoord tc = ph2 ? decode_tile(t - total1, p2.n_tiles, p.E, s_mt, s_off, G::PIECE)
                          : decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
@@ -728,7 +794,8 @@ cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
   if (err != cudaSuccess) return err;
   if constexpr (PAIR == 1) {
     const int grid = static_cast<int>(std::min<int64_t>(max_tiles, num_sms));
-    grouped_gemm_kernel<MODE, 1, false><<<grid, NUM_THREADS, smem, stream>>>(mapA, mapB, mapA, mapB, p, p, nullptr);
+    grouped_gemm_kernel<MODE, 1, false><<<grid, NUM_THREADS, smem, stream>>>(mapA, mapB, mapA, mapB, p, p, nullptr,
+                                                                              nullptr);
     return cudaGetLastError();
   } else {
     const int clusters =
@@ -746,7 +813,7 @@ cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 2, false>, mapA, mapB, mapA, mapB, p, p,
-                              static_cast<int*>(nullptr));
+                              static_cast<int*>(nullptr), static_cast<int*>(nullptr));
   }
 }
 
@@ -844,6 +911,11 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t stream) {
   return launch_with<MODE, 1>(mapA, mapB, p, a.num_sms, stream);
 }
 
+// Rows per expert at which one bf16 weight byte carries as many FLOPs (2 per
+// row per 2-byte weight) as the B200's measured bf16 peak per HBM byte
+// (about 1.66 PFLOP/s over 6.5 TB/s).
+constexpr int64_t kRidgeRowsPerExpert = 256;
+
 template <int MODE>
 cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down, int* arrivals,
                          cudaStream_t stream) {
@@ -874,7 +946,19 @@ cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down,
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 1, true>, mapA, mapB, mapA2, mapB2, p, p2, arrivals);
+  // The last counter is the tile scheduler's (pieces use the ones before it).
+  // Dynamic order pays where the weights stream from HBM (rows per expert
+  // below the bf16 ridge point of about 256 FLOP/byte), the static order
+  // where the tensor pipe bounds the launch; MOE_B200_TILE_SCHEDULE=dynamic
+  // or =static overrides the choice.
+  bool dynamic = up.R < kRidgeRowsPerExpert * up.E;
+  if (const char* env = std::getenv("MOE_B200_TILE_SCHEDULE")) {
+    if (env[0] == 'd') dynamic = true;
+    if (env[0] == 's') dynamic = false;
+  }
+  int* sched = dynamic ? arrivals + mega_ffn_counters(up.R, up.E) - 1 : nullptr;
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 1, true>, mapA, mapB, mapA2, mapB2, p, p2, arrivals,
+                            sched);
 }
 
 }  // namespace

@@ -84,7 +84,8 @@ cudaError_t launch_gemm_down(const GroupedGemmArgs& a, cudaStream_t stream);
 // which must not alias Xp).  A down tile of a 128-row piece waits (bounded)
 // until every gate_up tile of that piece has stored its h columns, counted
 // in arrivals[piece]; the counters must be zero at launch (launch_gather
-// clears them) and hold at least mega_ffn_counters(R, E) entries.
+// clears them) and hold at least mega_ffn_counters(R, E) entries: one per
+// possible 128-row piece, and last the tile scheduler's counter.
 int mega_ffn_counters(int R, int E);
 cudaError_t launch_mega_ffn(const GroupedGemmArgs& up, const GroupedGemmArgs& down, int* arrivals,
                             cudaStream_t stream);

@@ -38,8 +38,12 @@ def test_forward_small(name):
 # GEMM variants: both contractions in one cooperative launch (default), two
 # launches of one CTA per 128x256 tile, or two launches of a CTA pair per
 # 256x256 tile (tcgen05 cta_group::2); B stage tiles in one copy (default
-# where the column count allows) or in four 64-column copies.
-VARIANTS = {"single_launch": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1", "MOE_B200_B_ONE_BOX": "1"},
+# where the column count allows) or in four 64-column copies; the single
+# launch's tiles in static or dynamic (atomic counter) order.
+VARIANTS = {"single_launch": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1", "MOE_B200_B_ONE_BOX": "1",
+                              "MOE_B200_TILE_SCHEDULE": "static"},
+            "single_launch_dynamic": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1",
+                                      "MOE_B200_B_ONE_BOX": "1", "MOE_B200_TILE_SCHEDULE": "dynamic"},
             "single_launch_four_box": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1",
                                        "MOE_B200_B_ONE_BOX": "0"},
             "two_launches": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "1", "MOE_B200_B_ONE_BOX": "1"},
@@ -78,15 +82,18 @@ ALIGNED = {
 @pytest.mark.parametrize("name", sorted(SMALL) + sorted(ALIGNED))
 def test_single_launch_equals_two_launches(name, monkeypatch):
     """The single launch does the same tiles, MMAs and epilogues as the two
-    launches, only scheduled differently; a one-copy B stage tile has the same
+    launches, only scheduled differently (statically or from a tile counter);
+    a one-copy B stage tile has the same
     shared-memory image as four 64-column copies: every variant's output is
     identical bit for bit."""
     wl = SMALL.get(name) or ALIGNED[name]
     d = to_dev(make_inputs(wl, 11))
     outs = []
-    for single, one_box in (("1", "1"), ("0", "1"), ("1", "0"), ("0", "0")):
+    for single, one_box, order in (("1", "1", "static"), ("1", "1", "dynamic"), ("0", "1", "static"),
+                                   ("1", "0", "dynamic"), ("0", "0", "static")):
         monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", single)
         monkeypatch.setenv("MOE_B200_B_ONE_BOX", one_box)
+        monkeypatch.setenv("MOE_B200_TILE_SCHEDULE", order)
         run = GpuRun(wl, d)
         assert run.status == 0
         outs.append(run.out.clone())
