@@ -121,9 +121,19 @@ def test_forward_tiny_seeds(seed):
     dict(num_tokens=200, hidden_dim=8, moe_dim=8),              # single partial K block, tiny N
     dict(num_tokens=1100),                                      # R > 2048: separate router and CSR kernels
     dict(num_experts=600, num_tokens=40, logits_std=1.0),       # E > 512: separate router and CSR kernels
+    dict(num_experts=1024, top_k=32, num_tokens=40, logits_std=1.0),  # the library's largest E and k
+    dict(num_tokens=64, hidden_dim=8192, moe_dim=64),           # long gate_up K (128 K blocks), tiny down K
+    dict(num_tokens=48, hidden_dim=64, moe_dim=8192),           # long down K, 64 gate_up column blocks
 ])
 def test_forward_edge_cases(variant):
     run_and_check(WORKLOADS["tiny"].replace(**variant), seed=3)
+
+
+def test_sink_router_largest_shape():
+    """Sink router at its limits: 1024 routed experts, k + S = 32 lanes."""
+    wl = WORKLOADS["sink"].replace(num_tokens=50, hidden_dim=128, num_experts=1024, top_k=30, num_sink=2,
+                                   moe_dim=64)
+    run_and_check(wl, seed=9)
 
 
 def test_all_tokens_on_one_expert():
