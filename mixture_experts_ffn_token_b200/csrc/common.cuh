@@ -75,6 +75,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return false;
 }
 
+// ---------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may begin while
+// its predecessor on the stream is still finishing.  griddep_wait() blocks
+// until that predecessor has completed and its memory operations are visible
+// (a no-op for a kernel launched without it), so every kernel calls it before
+// its first global-memory access; griddep_launch_dependents() lets the next
+// such kernel begin launching before this one has finished.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------------- TMA
 // Tiled bulk tensor loads global -> this CTA's shared memory, completing on
 // an mbarrier (transaction bytes).  No multicast form is used anywhere.

@@ -16,6 +16,8 @@
 //           slot order and no atomic decides any position.
 #include <algorithm>
 
+#include <cstdlib>
+
 #include "kernels.cuh"
 
 namespace moe {
@@ -33,6 +35,8 @@ __device__ __forceinline__ bool slot_live(const uint8_t* mask, int64_t s, int k)
 __global__ void __launch_bounds__(kCsrThreads) csr_count_kernel(const int32_t* __restrict__ idx, int R, int E,
                                                                 int32_t* __restrict__ chunk_counts, int* status,
                                                                 const uint8_t* __restrict__ mask, int k) {
+  griddep_wait();  // the previous kernel's results are complete and visible
+  griddep_launch_dependents();
   extern __shared__ int cnt[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
@@ -54,6 +58,8 @@ __global__ void __launch_bounds__(kCsrThreads) csr_count_kernel(const int32_t* _
 __global__ void __launch_bounds__(1024) csr_scan_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int E,
                                                         int32_t* __restrict__ chunk_base,
                                                         int32_t* __restrict__ offsets) {
+  griddep_wait();  // the previous kernel's results are complete and visible
+  griddep_launch_dependents();
   __shared__ int warp_tot[32];
   const int e = threadIdx.x;
   const int lane = e & 31, warp = e >> 5;
@@ -98,6 +104,8 @@ __global__ void __launch_bounds__(kCsrThreads) csr_scatter_kernel(const int32_t*
                                                                   int32_t* __restrict__ perm,
                                                                   int32_t* __restrict__ inv,
                                                                   const uint8_t* __restrict__ mask, int k) {
+  griddep_wait();  // the previous kernel's results are complete and visible
+  griddep_launch_dependents();
   extern __shared__ int wcnt[];  // [kCsrWarps][E]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kCsrWarps * E; i += blockDim.x) wcnt[i] = 0;
@@ -145,6 +153,15 @@ __global__ void __launch_bounds__(kCsrThreads) csr_scatter_kernel(const int32_t*
   }
 }
 
+}  // namespace
+
+bool pdl_enabled() {
+  const char* env = std::getenv("MOE_B200_PDL");
+  return !(env != nullptr && env[0] == '0');
+}
+
+namespace {
+
 constexpr int kCombineBatch = 8;   // rows a combine thread loads before summing
 constexpr int kGatherUnroll = 4;   // 16-byte chunks a gather lane loads before storing
 
@@ -156,6 +173,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
                                                           int H, const float* __restrict__ scale,
                                                           __nv_bfloat16* __restrict__ Xp, int* status,
                                                           int* __restrict__ zero, int n_zero) {
+  griddep_wait();  // the previous kernel's results are complete and visible
+  griddep_launch_dependents();
   // Clear the caller's counters (the single-launch FFN's per-piece arrival
   // counts) for the kernel that follows on the stream.
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_zero; i += gridDim.x * blockDim.x) zero[i] = 0;
@@ -207,6 +226,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
                                                       const __nv_bfloat16* __restrict__ Ys, int Ns,
                                                       const uint8_t* __restrict__ mask,
                                                       __nv_bfloat16* __restrict__ out) {
+  griddep_wait();  // the previous kernel's results are complete and visible
+  griddep_launch_dependents();
   const int vec = H / 8;
   const int64_t n = static_cast<int64_t>(T) * vec;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
@@ -255,6 +276,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
 // slot space (so slot / Ns is the token and the gates are indexed by slot).
 __global__ void __launch_bounds__(256) shared_index_kernel(int T, int Ns, int32_t* __restrict__ offsets,
                                                            int32_t* __restrict__ perm) {
+  griddep_wait();  // the previous kernel's results are complete and visible
+  griddep_launch_dependents();
   const int64_t n = static_cast<int64_t>(T) * Ns;
   for (int64_t p = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; p < n;
        p += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -269,22 +292,20 @@ __global__ void __launch_bounds__(256) shared_index_kernel(int T, int Ns, int32_
 cudaError_t launch_shared_index(int T, int Ns, int32_t* offsets, int32_t* perm, int num_sms, cudaStream_t stream) {
   const int64_t n = static_cast<int64_t>(T) * Ns;
   const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, num_sms * 4)));
-  shared_index_kernel<<<blocks, 256, 0, stream>>>(T, Ns, offsets, perm);
-  return cudaGetLastError();
+  return launch_pdl(shared_index_kernel, dim3(blocks), dim3(256), 0, stream, T, Ns, offsets, perm);
 }
 
 cudaError_t launch_csr_count(const int32_t* idx, int R, int E, int32_t* chunk_counts, int* status,
                              const uint8_t* mask, int k, cudaStream_t stream) {
   const int nchunks = csr_num_chunks(R);
   if (nchunks == 0) return cudaSuccess;
-  csr_count_kernel<<<nchunks, kCsrThreads, E * sizeof(int), stream>>>(idx, R, E, chunk_counts, status, mask, k);
-  return cudaGetLastError();
+  return launch_pdl(csr_count_kernel, dim3(nchunks), dim3(kCsrThreads), E * sizeof(int), stream, idx, R, E,
+                    chunk_counts, status, mask, k);
 }
 
 cudaError_t launch_csr_scan(const int32_t* chunk_counts, int nchunks, int E, int32_t* chunk_base, int32_t* offsets,
                             cudaStream_t stream) {
-  csr_scan_kernel<<<1, 1024, 0, stream>>>(chunk_counts, nchunks, E, chunk_base, offsets);
-  return cudaGetLastError();
+  return launch_pdl(csr_scan_kernel, dim3(1), dim3(1024), 0, stream, chunk_counts, nchunks, E, chunk_base, offsets);
 }
 
 cudaError_t launch_csr_scatter(const int32_t* idx, int R, int E, const int32_t* chunk_base, int32_t* perm,
@@ -297,8 +318,8 @@ cudaError_t launch_csr_scatter(const int32_t* idx, int R, int E, const int32_t* 
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
   }
-  csr_scatter_kernel<<<nchunks, kCsrThreads, smem, stream>>>(idx, R, E, chunk_base, perm, inv, mask, k);
-  return cudaGetLastError();
+  return launch_pdl(csr_scatter_kernel, dim3(nchunks), dim3(kCsrThreads), smem, stream, idx, R, E, chunk_base, perm,
+                    inv, mask, k);
 }
 
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, const int32_t* offsets, int E, int R, int k,
@@ -308,8 +329,8 @@ cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, const int
   const int rows_per_block = 8;
   const int blocks = static_cast<int>(std::min<int64_t>((R + rows_per_block - 1) / rows_per_block,
                                                         static_cast<int64_t>(num_sms) * 16));
-  gather_rows_kernel<<<blocks, 256, 0, stream>>>(x, perm, offsets, E, R, k, H, scale, Xp, status, zero, n_zero);
-  return cudaGetLastError();
+  return launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, stream, x, perm, offsets, E, R, k, H, scale, Xp,
+                    status, zero, n_zero);
 }
 
 cudaError_t launch_combine(const __nv_bfloat16* Y, int T, int H, int k, const __nv_bfloat16* Ys, int Ns,
@@ -317,8 +338,7 @@ cudaError_t launch_combine(const __nv_bfloat16* Y, int T, int H, int k, const __
   if (T == 0) return cudaSuccess;
   const int64_t n = static_cast<int64_t>(T) * (H / 8);
   const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(num_sms) * 16));
-  combine_kernel<<<blocks, 256, 0, stream>>>(Y, T, H, k, Ys, Ns, mask, out);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(blocks), dim3(256), 0, stream, Y, T, H, k, Ys, Ns, mask, out);
 }
 
 }  // namespace moe

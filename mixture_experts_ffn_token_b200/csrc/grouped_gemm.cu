@@ -413,6 +413,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_relinquish();
     }
   }
+  griddep_wait();  // the CSR and operands of the kernels before are complete and visible
   for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) s_off[i] = p.offsets[i];
   __syncthreads();
   if (warp == 0) {
@@ -694,6 +695,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 
   __syncthreads();
+  griddep_launch_dependents();  // this CTA has no tiles left: the next kernel may begin launching
   if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, p.err_bit);
   if constexpr (PAIR == 2) {
     tc_fence_before_sync();

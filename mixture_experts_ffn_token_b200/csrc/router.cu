@@ -124,6 +124,8 @@ __device__ __forceinline__ int route_token(const RouterArgs& a, int t, int lane)
 
 template <int NPL, bool SINK, bool BF16>
 __global__ void __launch_bounds__(128) router_kernel(const RouterArgs a) {
+  griddep_wait();  // the previous kernel's results are complete and visible
+  griddep_launch_dependents();
   if (a.status_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.status_reset = 0;
   const int lane = threadIdx.x & 31;
   const int t = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
@@ -140,6 +142,8 @@ template <int NPL, bool SINK, bool BF16>
 __global__ void __launch_bounds__(32 * kSmallWarps) route_csr_small_kernel(const RouterArgs a, int32_t* offsets,
                                                                            int32_t* perm, int* status,
                                                                            const uint8_t* mask) {
+  griddep_wait();  // the previous kernel's results are complete and visible
+  griddep_launch_dependents();
   extern __shared__ int sm[];
   int* s_idx = sm;                           // [R]
   int* wcnt = sm + kSmallSlots;              // [kSmallWarps][E]
@@ -227,13 +231,11 @@ cudaError_t launch_npl(const RouterArgs& a, cudaStream_t stream) {
   const dim3 grid((a.T + warps_per_block - 1) / warps_per_block);
   const dim3 block(32 * warps_per_block);
   if (a.sink) {
-    if (a.logits_bf16) router_kernel<NPL, true, true><<<grid, block, 0, stream>>>(a);
-    else router_kernel<NPL, true, false><<<grid, block, 0, stream>>>(a);
-  } else {
-    if (a.logits_bf16) router_kernel<NPL, false, true><<<grid, block, 0, stream>>>(a);
-    else router_kernel<NPL, false, false><<<grid, block, 0, stream>>>(a);
+    if (a.logits_bf16) return launch_pdl(router_kernel<NPL, true, true>, grid, block, 0, stream, a);
+    return launch_pdl(router_kernel<NPL, true, false>, grid, block, 0, stream, a);
   }
-  return cudaGetLastError();
+  if (a.logits_bf16) return launch_pdl(router_kernel<NPL, false, true>, grid, block, 0, stream, a);
+  return launch_pdl(router_kernel<NPL, false, false>, grid, block, 0, stream, a);
 }
 
 template <int NPL>
@@ -241,14 +243,15 @@ cudaError_t launch_small_npl(const RouterArgs& a, int32_t* offsets, int32_t* per
                              const uint8_t* mask, cudaStream_t stream) {
   const size_t smem = (kSmallSlots + static_cast<size_t>(kSmallWarps) * a.E) * sizeof(int);
   const dim3 block(32 * kSmallWarps);
+  const dim3 one(1);
   if (a.sink) {
-    if (a.logits_bf16) route_csr_small_kernel<NPL, true, true><<<1, block, smem, stream>>>(a, offsets, perm, status, mask);
-    else route_csr_small_kernel<NPL, true, false><<<1, block, smem, stream>>>(a, offsets, perm, status, mask);
-  } else {
-    if (a.logits_bf16) route_csr_small_kernel<NPL, false, true><<<1, block, smem, stream>>>(a, offsets, perm, status, mask);
-    else route_csr_small_kernel<NPL, false, false><<<1, block, smem, stream>>>(a, offsets, perm, status, mask);
+    if (a.logits_bf16)
+      return launch_pdl(route_csr_small_kernel<NPL, true, true>, one, block, smem, stream, a, offsets, perm, status, mask);
+    return launch_pdl(route_csr_small_kernel<NPL, true, false>, one, block, smem, stream, a, offsets, perm, status, mask);
   }
-  return cudaGetLastError();
+  if (a.logits_bf16)
+    return launch_pdl(route_csr_small_kernel<NPL, false, true>, one, block, smem, stream, a, offsets, perm, status, mask);
+  return launch_pdl(route_csr_small_kernel<NPL, false, false>, one, block, smem, stream, a, offsets, perm, status, mask);
 }
 
 }  // namespace

@@ -101,6 +101,22 @@ def test_single_launch_equals_two_launches(name, monkeypatch):
         assert torch.equal(outs[0], o)
 
 
+@pytest.mark.parametrize("name", ["tiny", "sink_small", "gptoss_small"])
+def test_programmatic_launch_changes_nothing(name, monkeypatch):
+    """Kernels launched to overlap their predecessor's tail (programmatic
+    dependent launch) wait for its results first: the same bits either way."""
+    wl = SMALL[name]
+    d = to_dev(make_inputs(wl, 13))
+    outs = []
+    for pdl in ("1", "0"):
+        monkeypatch.setenv("MOE_B200_PDL", pdl)
+        run = GpuRun(wl, d)
+        assert run.status == 0
+        outs.append((run.out.clone(), run.idx.clone(), run.w.clone()))
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b)
+
+
 @pytest.mark.parametrize("name", sorted(ALIGNED))
 def test_one_box_layouts_against_oracle(name, monkeypatch):
     monkeypatch.setenv("MOE_B200_B_ONE_BOX", "1")
