@@ -48,7 +48,7 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t stream);
 
 // Routing plus the whole CSR build (offsets, permutation) in one CTA, for
 // problems with at most kSmallSlots routed slots and kSmallExperts experts.
-constexpr int kSmallWarps = 16;
+constexpr int kSmallWarps = 32;
 constexpr int kSmallSlots = 2048;
 constexpr int kSmallExperts = 512;
 cudaError_t launch_route_csr_small(const RouterArgs& a, int32_t* offsets, int32_t* perm, int* status,

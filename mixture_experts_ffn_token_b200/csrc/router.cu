@@ -244,6 +244,24 @@ cudaError_t launch_small_npl(const RouterArgs& a, int32_t* offsets, int32_t* per
   const size_t smem = (kSmallSlots + static_cast<size_t>(kSmallWarps) * a.E) * sizeof(int);
   const dim3 block(32 * kSmallWarps);
   const dim3 one(1);
+  // the per-warp histograms need up to (2048 + 32 * 512) * 4 bytes, above the default 48 KB
+  static bool opted_in = false;
+  if (!opted_in) {
+    const int max_smem = static_cast<int>((kSmallSlots + static_cast<size_t>(kSmallWarps) * kSmallExperts) * sizeof(int));
+    cudaError_t e =
+        cudaFuncSetAttribute(route_csr_small_kernel<NPL, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(route_csr_small_kernel<NPL, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               max_smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(route_csr_small_kernel<NPL, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               max_smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(route_csr_small_kernel<NPL, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               max_smem);
+    if (e != cudaSuccess) return e;
+    opted_in = true;
+  }
   if (a.sink) {
     if (a.logits_bf16)
       return launch_pdl(route_csr_small_kernel<NPL, true, true>, one, block, smem, stream, a, offsets, perm, status, mask);
