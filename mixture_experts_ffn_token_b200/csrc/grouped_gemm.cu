@@ -551,7 +551,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // CTA loads its 128 rows of A and its half of the 256 columns.
             if (leader) mbar_arrive_expect_tx(full0 + 8 * s, 2 * G::STAGE_BYTES);
             tma_load_2d_pair(sa, &mapA, fb, kc, arow);
-            if constexpr (MODE == MODE_GATE_UP_CONCAT) {
+            if (p.b_one_box) {
+              // this CTA's two 64-column blocks in one copy (concatenated:
+              // the leader's gate half, the peer's up half)
+              if constexpr (MODE == MODE_GATE_UP_CONCAT)
+                tma_load_5d_pair(sb, &mapB, fb, 0, kc, 2 * tc.n, static_cast<int>(rank), tc.e);
+              else
+                tma_load_4d_pair(sb, &mapB, fb, 0, kc, 4 * tc.n + 2 * static_cast<int>(rank), tc.e);
+            } else if constexpr (MODE == MODE_GATE_UP_CONCAT) {
               // leader: the 128 gate columns; peer: the matching 128 up columns
               const int c0 = tc.n * 128;
               const int half = static_cast<int>(rank);
@@ -827,33 +834,34 @@ cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
 // depends only on the shared address).  Requires the columns of one half to
 // be a multiple of 64, so that every in-range coordinate stays inside the
 // tensor; otherwise (or if the driver declines the view) false.
+// `pair`: a CTA of a pair loads half of the 256 columns (2 blocks; the
+// concatenated view then holds one of the gate/up halves per copy).
 template <int MODE>
-bool encode_one_box_b(const GroupedGemmArgs& a, CUtensorMap* map) {
+bool encode_one_box_b(const GroupedGemmArgs& a, CUtensorMap* map, bool pair) {
   const cuuint64_t H = a.H, D = a.D, E = a.E;
   if (MODE == MODE_GATE_UP_CONCAT) {
     if (D % 64 != 0) return false;
     const cuuint64_t dims[5] = {64, H, D / 64, 2, E};
     const cuuint64_t strides[4] = {2 * D * 2, 128, D * 2, H * 2 * D * 2};
-    const cuuint32_t box[5] = {64, BK, 2, 2, 1};
+    const cuuint32_t box[5] = {64, BK, 2, pair ? 1u : 2u, 1};
     return encode_bf16_map(map, a.W, 5, dims, strides, box);
   } else if (MODE == MODE_GATE_UP_INTERLEAVED) {
     if ((2 * D) % 64 != 0) return false;
     const cuuint64_t dims[4] = {64, H, 2 * D / 64, E};
     const cuuint64_t strides[3] = {2 * D * 2, 128, H * 2 * D * 2};
-    const cuuint32_t box[4] = {64, BK, 4, 1};
+    const cuuint32_t box[4] = {64, BK, pair ? 2u : 4u, 1};
     return encode_bf16_map(map, a.W, 4, dims, strides, box);
   } else {
     if (H % 64 != 0) return false;
     const cuuint64_t dims[4] = {64, D, H / 64, E};
     const cuuint64_t strides[3] = {H * 2, 128, D * H * 2};
-    const cuuint32_t box[4] = {64, BK, 4, 1};
+    const cuuint32_t box[4] = {64, BK, pair ? 2u : 4u, 1};
     return encode_bf16_map(map, a.W, 4, dims, strides, box);
   }
 }
 
 template <int MODE>
-cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& mapB, GemmParams& p,
-                    bool allow_one_box) {
+cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& mapB, GemmParams& p, bool pair) {
   const bool down = MODE == MODE_DOWN;
   const int K = down ? a.D : a.H;
   {
@@ -863,7 +871,7 @@ cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& ma
     if (!encode_bf16_map(&mapA, a.A, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
   const cuuint64_t H = a.H, D = a.D, E = a.E;
-  p.b_one_box = allow_one_box && one_box_enabled() && encode_one_box_b<MODE>(a, &mapB) ? 1 : 0;
+  p.b_one_box = one_box_enabled() && encode_one_box_b<MODE>(a, &mapB, pair) ? 1 : 0;
   if (p.b_one_box) {
     // mapB already holds the one-copy view
   } else if (MODE == MODE_GATE_UP_CONCAT) {
@@ -907,7 +915,7 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t stream) {
   CUtensorMap mapA, mapB;
   GemmParams p;
   const int pair = choose_pair(a.R, a.E);
-  cudaError_t err = prepare<MODE>(a, mapA, mapB, p, pair == 1);
+  cudaError_t err = prepare<MODE>(a, mapA, mapB, p, pair == 2);
   if (err != cudaSuccess) return err;
   if (pair == 2) return launch_with<MODE, 2>(mapA, mapB, p, a.num_sms, stream);
   return launch_with<MODE, 1>(mapA, mapB, p, a.num_sms, stream);
@@ -924,9 +932,9 @@ cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down,
   if (up.R == 0) return cudaSuccess;
   CUtensorMap mapA, mapB, mapA2, mapB2;
   GemmParams p, p2;
-  cudaError_t err = prepare<MODE>(up, mapA, mapB, p, true);
+  cudaError_t err = prepare<MODE>(up, mapA, mapB, p, false);
   if (err != cudaSuccess) return err;
-  err = prepare<MODE_DOWN>(down, mapA2, mapB2, p2, true);
+  err = prepare<MODE_DOWN>(down, mapA2, mapB2, p2, false);
   if (err != cudaSuccess) return err;
   // a timeout anywhere in the fused launch is reported as both stages'
   p.err_bit = p2.err_bit = MOE_DEVICE_ERR_TIMEOUT_GEMM1 | MOE_DEVICE_ERR_TIMEOUT_GEMM2;

@@ -101,6 +101,23 @@ def test_single_launch_equals_two_launches(name, monkeypatch):
         assert torch.equal(outs[0], o)
 
 
+@pytest.mark.parametrize("name", sorted(ALIGNED))
+def test_cta_pair_one_copy_equals_two_copies(name, monkeypatch):
+    """In the CTA-pair variant each CTA's 128-column half of B arrives in one
+    copy or in two 64-column copies: the same shared-memory image, the same bits."""
+    wl = ALIGNED[name]
+    d = to_dev(make_inputs(wl, 14))
+    monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", "0")
+    monkeypatch.setenv("MOE_B200_CTA_PAIR", "2")
+    outs = []
+    for one_box in ("1", "0"):
+        monkeypatch.setenv("MOE_B200_B_ONE_BOX", one_box)
+        run = GpuRun(wl, d)
+        assert run.status == 0
+        outs.append(run.out.clone())
+    assert torch.equal(outs[0], outs[1])
+
+
 @pytest.mark.parametrize("name", ["tiny", "sink_small", "gptoss_small"])
 def test_programmatic_launch_changes_nothing(name, monkeypatch):
     """Kernels launched to overlap their predecessor's tail (programmatic
