@@ -17,6 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
 
 MOE_OK = 0
+MOE_ERR_DEVICE_TIMEOUT = 5
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARGUMENT", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT"}
 ROUTERS = {"softmax_topk": 0, "sigmoid_sink": 1}
@@ -278,6 +279,6 @@ def moe_device_status(workspace, stream=None) -> int:
     """The device fault bits recorded in the workspace (synchronizes the stream)."""
     v = ctypes.c_int32(0)
     st = load_library().moe_device_status(_p(workspace), ctypes.byref(v), _stream(stream))
-    if st not in (MOE_OK, 5):
+    if st not in (MOE_OK, MOE_ERR_DEVICE_TIMEOUT):
         raise MoEError(st, "moe_device_status")
     return v.value

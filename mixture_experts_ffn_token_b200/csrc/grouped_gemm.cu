@@ -97,6 +97,11 @@ struct GemmParams {
   float alpha, limit;
   int err_bit;
   int b_one_box;  // 1: the B tensor map delivers a stage's whole B tile in one copy
+  // single launch: arrivals a down tile waits for beyond the real ones (0; 1
+  // only under the test hook, which then never completes) and the time limit
+  // of that wait
+  int extra_arrivals;
+  unsigned long long dep_timeout_ns;
 };
 
 struct TileCoord {
@@ -178,7 +183,7 @@ __device__ __forceinline__ bool ring_take(uint32_t ring_full0, uint32_t ring_emp
 // err bits recorded at once so other CTAs stop waiting too) after the
 // timeout, when this CTA aborts, or when another CTA has recorded a timeout.
 __device__ __forceinline__ bool wait_arrivals(const int* counter, int target, volatile int* abort,
-                                              volatile int* status, int err_bits) {
+                                              volatile int* status, int err_bits, uint64_t timeout_ns) {
   if (ld_acquire(counter) >= target) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1; it < (1u << 26); ++it) {
@@ -186,7 +191,7 @@ __device__ __forceinline__ bool wait_arrivals(const int* counter, int target, vo
     if (ld_acquire(counter) >= target) return true;
     if ((it & 15u) == 0) {
       if (*abort || (*status & err_bits) != 0) break;
-      if (global_timer_ns() - t0 > kTimeoutNs) break;
+      if (global_timer_ns() - t0 > timeout_ns) break;
     }
   }
   *abort = 1;
@@ -459,7 +464,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int tile_stride = gridDim.x / PAIR;
   // down tiles of a piece wait for this many arrivals (one per epilogue warp
   // of each of the piece's gate_up tiles)
-  const int arrivals_needed = NUM_EPI_WARPS * p.n_tiles;
+  const int arrivals_needed = NUM_EPI_WARPS * p.n_tiles + p.extra_arrivals;
   const bool dyn = FUSED && sched != nullptr;  // dynamic tile order
 
   if (warp == 0) {
@@ -493,7 +498,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int nkb = ph2 ? p2.num_kb : p.num_kb;
         if constexpr (FUSED) {
           if (ph2) {
-            if (!wait_arrivals(arrivals + tc.piece, arrivals_needed, abort_flag, p.status, p.err_bit)) {
+            if (!wait_arrivals(arrivals + tc.piece, arrivals_needed, abort_flag, p.status, p.err_bit,
+                               p.dep_timeout_ns)) {
               ok = false;
               break;
             }
@@ -872,6 +878,19 @@ cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& ma
   }
   const cuuint64_t H = a.H, D = a.D, E = a.E;
   p.b_one_box = one_box_enabled() && encode_one_box_b<MODE>(a, &mapB, pair) ? 1 : 0;
+  // Test hook for the single launch's bounded cross-CTA wait:
+  // MOE_B200_TEST_STALL_DOWN_TILES_MS=<ms> makes every down tile wait for one
+  // arrival more than will ever come, giving up after <ms>; the launch then
+  // records MOE_DEVICE_ERR_TIMEOUT_GEMM1 | _GEMM2 and ends normally.
+  p.extra_arrivals = 0;
+  p.dep_timeout_ns = kTimeoutNs;
+  if (const char* env = std::getenv("MOE_B200_TEST_STALL_DOWN_TILES_MS")) {
+    const long ms = std::strtol(env, nullptr, 10);
+    if (ms > 0) {
+      p.extra_arrivals = 1;
+      p.dep_timeout_ns = static_cast<unsigned long long>(std::min(ms, 2000L)) * 1000000ull;
+    }
+  }
   if (p.b_one_box) {
     // mapB already holds the one-copy view
   } else if (MODE == MODE_GATE_UP_CONCAT) {
