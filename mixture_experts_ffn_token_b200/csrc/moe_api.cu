@@ -5,6 +5,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kernels.cuh"
 
 using moe::kMaxExperts;
@@ -203,6 +205,29 @@ moe::RouterArgs router_args(const moe_config_t* c, const void* logits, const flo
 }
 
 // Records ev[i] on the stream when events are requested.
+// NVTX ranges (MOE_B200_NVTX=1): one per API call and one around the
+// enqueue of each kernel, named "moe.<stage>", for a timeline profiler to
+// line up with the kernels.  Off by default (no NVTX call is made).
+bool nvtx_enabled() {
+  static const bool on = [] {
+    const char* env = std::getenv("MOE_B200_NVTX");
+    return env != nullptr && env[0] == '1';
+  }();
+  return on;
+}
+
+struct NvtxRange {
+  const bool on;
+  explicit NvtxRange(const char* name) : on(nvtx_enabled()) {
+    if (on) nvtxRangePushA(name);
+  }
+  ~NvtxRange() {
+    if (on) nvtxRangePop();
+  }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 struct Recorder {
   cudaEvent_t const* ev;
   cudaStream_t stream;
@@ -227,10 +252,13 @@ moe_status_t enqueue_grouped_pass(const moe_config_t* c, int E, int k, int D, co
   const int R = T * k;
   const bool fused = single_launch();
   rec(base);
-  if (moe::launch_gather(static_cast<const __nv_bfloat16*>(x), perm, offsets, E, R, k, H, scale, xp, status,
-                         num_sms, stream, fused ? arr : nullptr, fused ? moe::mega_ffn_counters(R, E) : 0) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
+  {
+    const NvtxRange range("moe.gather");
+    if (moe::launch_gather(static_cast<const __nv_bfloat16*>(x), perm, offsets, E, R, k, H, scale, xp, status,
+                           num_sms, stream, fused ? arr : nullptr, fused ? moe::mega_ffn_counters(R, E) : 0) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   moe::GroupedGemmArgs g;
   g.offsets = offsets;
   g.perm = perm;
@@ -259,13 +287,22 @@ moe_status_t enqueue_grouped_pass(const moe_config_t* c, int E, int k, int D, co
   *y_out = g2.out;
   rec(base + 1);
   if (fused) {
-    if (moe::launch_mega_ffn(g, g2, arr, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    {
+      const NvtxRange range("moe.mega_ffn");
+      if (moe::launch_mega_ffn(g, g2, arr, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    }
     rec(base + 2);
     return MOE_OK;
   }
-  if (moe::launch_gemm_gate_up(g, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    const NvtxRange range("moe.gemm_gate_up");
+    if (moe::launch_gemm_gate_up(g, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  }
   rec(base + 2);
-  if (moe::launch_gemm_down(g2, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    const NvtxRange range("moe.gemm_down");
+    if (moe::launch_gemm_down(g2, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  }
   return MOE_OK;
 }
 
@@ -285,9 +322,12 @@ moe_status_t enqueue_ffn(const moe_config_t* c, const void* x, const void* gate_
                                          num_sms, stream, rec, 0);
   if (st != MOE_OK) return st;
   rec(3);
-  if (moe::launch_combine(y, c->num_tokens, c->hidden_dim, c->top_k, nullptr, 0, nullptr,
-                          static_cast<__nv_bfloat16*>(out), num_sms, stream) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  {
+    const NvtxRange range("moe.combine");
+    if (moe::launch_combine(y, c->num_tokens, c->hidden_dim, c->top_k, nullptr, 0, nullptr,
+                            static_cast<__nv_bfloat16*>(out), num_sms, stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   rec(4);
   return MOE_OK;
 }
@@ -298,17 +338,26 @@ moe_status_t enqueue_csr(const moe_config_t* c, const int32_t* idx, int32_t* off
   const int R = c->num_tokens * c->top_k, E = c->num_experts, k = c->top_k;
   const Recorder rec{ev, stream};
   rec(0);
-  if (moe::launch_csr_count(idx, R, E, at<int32_t>(ws, L.chunk_counts), at<int>(ws, L.status), mask, k, stream) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
+  {
+    const NvtxRange range("moe.csr_count");
+    if (moe::launch_csr_count(idx, R, E, at<int32_t>(ws, L.chunk_counts), at<int>(ws, L.status), mask, k, stream) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   rec(1);
-  if (moe::launch_csr_scan(at<int32_t>(ws, L.chunk_counts), moe::csr_num_chunks(R), E, at<int32_t>(ws, L.chunk_base),
-                           offsets, stream) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  {
+    const NvtxRange range("moe.csr_scan");
+    if (moe::launch_csr_scan(at<int32_t>(ws, L.chunk_counts), moe::csr_num_chunks(R), E, at<int32_t>(ws, L.chunk_base),
+                             offsets, stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   rec(2);
-  if (moe::launch_csr_scatter(idx, R, E, at<int32_t>(ws, L.chunk_base), perm, inv, mask, k, stream) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
+  {
+    const NvtxRange range("moe.csr_scatter");
+    if (moe::launch_csr_scatter(idx, R, E, at<int32_t>(ws, L.chunk_base), perm, inv, mask, k, stream) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   return MOE_OK;
 }
 
@@ -350,6 +399,7 @@ moe_status_t forward_impl(const moe_config_t* cfg, const moe_extras_t* extras, c
                           const void* gate_up_b, const void* down_w, const void* down_b, void* out, int32_t* idx_out,
                           float* w_out, float* sink_out, void* ws, size_t ws_bytes, cudaStream_t stream,
                           cudaEvent_t const* ev) {
+  const NvtxRange api_range("moe_forward");
   moe_status_t st = validate_config(cfg);
   if (st != MOE_OK) return st;
   Extras ex;
@@ -380,11 +430,17 @@ moe_status_t forward_impl(const moe_config_t* cfg, const moe_extras_t* extras, c
     // small (decode-sized) problems: routing and the CSR build in one CTA;
     // the CSR stages then record back-to-back events
     const moe::RouterArgs ra = router_args(cfg, logits, expert_bias, global_scale, idx, w, sink, nullptr);
-    if (moe::launch_route_csr_small(ra, offsets, perm, status, ex.mask, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    {
+      const NvtxRange range("moe.route_csr_small");
+      if (moe::launch_route_csr_small(ra, offsets, perm, status, ex.mask, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    }
     for (int i = 1; i <= 3; ++i) rec(i);
   } else {
     const moe::RouterArgs ra = router_args(cfg, logits, expert_bias, global_scale, idx, w, sink, status);
-    if (moe::launch_router(ra, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    {
+      const NvtxRange range("moe.router");
+      if (moe::launch_router(ra, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    }
     if ((st = enqueue_csr(cfg, idx, offsets, perm, nullptr, ws, L, stream, ev != nullptr ? ev + 1 : nullptr,
                           ex.mask)) != MOE_OK)
       return st;
@@ -407,7 +463,10 @@ moe_status_t forward_impl(const moe_config_t* cfg, const moe_extras_t* extras, c
     // weights (sink router) or by 1
     int32_t* s_off = at<int32_t>(ws, L.sh_offsets);
     int32_t* s_perm = at<int32_t>(ws, L.sh_perm);
-    if (moe::launch_shared_index(T, ex.Ns, s_off, s_perm, num_sms, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    {
+      const NvtxRange range("moe.shared_index");
+      if (moe::launch_shared_index(T, ex.Ns, s_off, s_perm, num_sms, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    }
     const float* gates = cfg->router == MOE_ROUTER_SIGMOID_SINK ? sink : nullptr;
     st = enqueue_grouped_pass(cfg, ex.Ns, ex.Ns, ex.Ds, x, ex.s_gu_w, ex.s_gu_b, ex.s_d_w, ex.s_d_b, s_off, s_perm,
                               ex.weight_first ? gates : nullptr, ex.weight_first ? nullptr : gates,
@@ -419,9 +478,12 @@ moe_status_t forward_impl(const moe_config_t* cfg, const moe_extras_t* extras, c
     for (int i = 8; i <= 10; ++i) rec(i);
   }
   rec(11);
-  if (moe::launch_combine(y, T, cfg->hidden_dim, k, ys, ex.Ns, ex.mask, static_cast<__nv_bfloat16*>(out), num_sms,
-                          stream) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  {
+    const NvtxRange range("moe.combine");
+    if (moe::launch_combine(y, T, cfg->hidden_dim, k, ys, ex.Ns, ex.mask, static_cast<__nv_bfloat16*>(out), num_sms,
+                            stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   rec(12);
   return MOE_OK;
 }
@@ -459,6 +521,7 @@ moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
 moe_status_t moe_route(const moe_config_t* cfg, const void* logits, const float* expert_bias,
                        const float* global_scale, int32_t* expert_indices, float* expert_weights,
                        float* sink_weights, moe_stream_t stream) {
+  const NvtxRange api_range("moe_route");
   moe_status_t st = validate_config(cfg);
   if (st != MOE_OK) return st;
   if (cfg->num_tokens == 0) return MOE_OK;
@@ -475,6 +538,7 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* logits, const float*
 moe_status_t moe_create_indices(const moe_config_t* cfg, const int32_t* expert_indices, int32_t* expert_offsets,
                                 int32_t* permutation, int32_t* inverse, void* workspace, size_t workspace_bytes,
                                 moe_stream_t stream) {
+  const NvtxRange api_range("moe_create_indices");
   moe_status_t st = validate_config(cfg);
   if (st != MOE_OK) return st;
   if (expert_offsets == nullptr) return MOE_ERR_INVALID_ARGUMENT;
@@ -492,6 +556,7 @@ moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x, const void*
                              const void* down_w, const void* down_b, const int32_t* expert_offsets,
                              const int32_t* permutation, const float* expert_weights, void* out, void* workspace,
                              size_t workspace_bytes, moe_stream_t stream) {
+  const NvtxRange api_range("moe_grouped_ffn");
   moe_status_t st = validate_config(cfg);
   if (st != MOE_OK) return st;
   if (cfg->num_tokens == 0) return MOE_OK;

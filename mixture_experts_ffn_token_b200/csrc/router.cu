@@ -39,16 +39,25 @@ __device__ __forceinline__ float load_logit(const void* logits, int64_t i) {
 
 __device__ __forceinline__ double log_sigmoid(double z) { return fmin(z, 0.0) - log1p(exp(-fabs(z))); }
 
+// Order-preserving unsigned image of a float score: a > b exactly when
+// key(a) > key(b), with -0 taken as +0 (they compare equal) and NaN mapped to
+// 0, below every number (-inf included), so a NaN score is never selected.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  if (v != v) return 0u;
+  const uint32_t b = __float_as_uint(v == 0.f ? 0.f : v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
 // Routes token t with the calling warp; returns this lane's selected expert
 // (lanes 0..k-1, in selection order) and writes idx, w and sink_w.
 template <int NPL, bool SINK, bool BF16>
 __device__ __forceinline__ int route_token(const RouterArgs& a, int t, int lane) {
   const int64_t row = static_cast<int64_t>(t) * a.stride;
-  float key[NPL];
+  uint32_t key[NPL];  // order_key of each score, 0 = not selectable
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
     const int e = lane + 32 * i;
-    float kv = -INFINITY;
+    float kv = NAN;
     if (e < a.E) {
       const float z = load_logit<BF16>(a.logits, row + e);
       if constexpr (SINK) {
@@ -59,35 +68,30 @@ __device__ __forceinline__ int route_token(const RouterArgs& a, int t, int lane)
         kv = z;
       }
     }
-    key[i] = kv;
+    key[i] = order_key(kv);
   }
 
+  // k rounds: the largest remaining key over the warp (one redux), then the
+  // lowest expert index holding it (a second redux) -- ties go to the lowest
+  // index, as the oracle decides them.
   uint32_t taken = 0;
   int my_e = 0;
   for (int j = 0; j < a.k; ++j) {
-    float bv = -INFINITY;
+    uint32_t bv = 0;
     int bi = INT_MAX;
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
-      const int e = lane + 32 * i;
-      if (e < a.E && !((taken >> i) & 1u)) {
-        if (key[i] > bv || (key[i] == bv && e < bi)) {
-          bv = key[i];
-          bi = e;
-        }
+      // e grows with i, so a strict > keeps the lowest index among equal keys
+      if (!((taken >> i) & 1u) && key[i] > bv) {
+        bv = key[i];
+        bi = lane + 32 * i;
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    // bi == INT_MAX only for NaN scores: the index is then left out of range
-    // and the CSR build flags it.
+    const uint32_t best = __reduce_max_sync(0xffffffffu, bv);
+    const int cand = (best != 0u && bv == best) ? bi : INT_MAX;
+    bi = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<uint32_t>(cand)));
+    // bi == INT_MAX only when no selectable score is left (NaN scores): the
+    // index is then out of range and the CSR build flags it.
     if (bi < a.E && (bi & 31) == lane) taken |= 1u << (bi >> 5);
     if (lane == j) my_e = bi;
   }

@@ -209,6 +209,10 @@ def test_softmax_router(E, k, logits_dtype):
     g = torch.Generator().manual_seed(E * 7 + k)
     logits = (torch.randn(T, E, generator=g) * 2).to(logits_dtype)
     logits[7, :] = 0.5                    # all ties: lowest indices, in order
+    logits[9, :] = float("-inf")          # one finite logit, then -inf ties by lowest index
+    logits[9, E // 2] = 1.0
+    logits[10, :] = 0.0                   # +0 and -0 compare equal: lowest indices
+    logits[10, 1::2] = -0.0
     wl = WORKLOADS["tiny"].replace(num_experts=E, top_k=k, num_tokens=T)
     cfg = abi.make_config(wl, logits_dtype=logits_dtype)
     idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
@@ -219,6 +223,8 @@ def test_softmax_router(E, k, logits_dtype):
     i_ref, w_ref = oracle.route_softmax_topk(host, E, k)
     assert np.array_equal(idx.cpu().numpy(), i_ref)
     assert idx[7].tolist() == list(range(k))
+    assert idx[10].tolist() == list(range(k))
+    assert idx[9, 0].item() == E // 2
     check_weights(w.cpu().numpy(), w_ref)
 
 
@@ -353,3 +359,21 @@ def test_forward_full_size_sampled(name):
     rng = np.random.default_rng(123)
     sample = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=min(T, FULL_SAMPLE), replace=False)]))
     run_and_check(wl, seed=0, device_inputs=True, sample_tokens=sample)
+
+
+def test_nvtx_ranges_change_nothing():
+    """With MOE_B200_NVTX=1 (read once per process) every API call and kernel
+    enqueue is wrapped in an NVTX range; the layer still matches the oracle."""
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    script = ("import sys; sys.path.insert(0, %r); sys.path.insert(0, %r)\n"
+              "from gpu_helpers import run_and_check\n"
+              "from test_gpu_parity import SMALL\n"
+              "run_and_check(SMALL['sink_small'], seed=15)\n"
+              "run_and_check(SMALL['decode_small'], seed=15)\n"
+              "print('ok')\n") % (here, os.path.dirname(here))
+    env = dict(os.environ, MOE_B200_NVTX="1")
+    r = subprocess.run([sys.executable, "-c", script], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stderr[-2000:]
