@@ -15,7 +15,7 @@
 // Design: the page's kernel uses one block per token and one thread per
 // expert with a block-level top-k.  Here one warp owns a token: each lane
 // holds ceil(E/32) scores in registers, the k winners are found by k rounds
-// of a 5-step shuffle arg-max (ties -> lower index), and lanes 0..k+S-1 then
+// of two warp reductions (ties -> lower index), and lanes 0..k+S-1 then
 // hold one normalisation entry each, so the final softmax is one warp
 // reduction.  The selection score is the fp32 value fl32(sigmoid(z)) + b
 // (sigmoid evaluated in fp64 and rounded once), so the choice is decided in
