@@ -137,26 +137,41 @@ def load_library():
     return lib
 
 
+def config(num_tokens: int, hidden_dim: int, num_experts: int, top_k: int, moe_dim: int, *,
+           router: str = "softmax_topk", num_sink: int = 0, logits_dtype=torch.float32,
+           logits_row_stride: Optional[int] = None, route_scale: float = 1.0,
+           gate_up_format: str = "concatenated", activation: str = "silu", alpha: float = 0.0,
+           limit: float = 0.0, has_bias: bool = False) -> MoEConfig:
+    """moe_config_t from keyword arguments (names as in include/moe.h; router
+    "softmax_topk" | "sigmoid_sink", gate_up_format "concatenated" |
+    "interleaved", activation "silu" | "swigluoai" | "gelu_tanh")."""
+    c = MoEConfig()
+    c.num_tokens = num_tokens
+    c.hidden_dim = hidden_dim
+    c.num_experts = num_experts
+    c.top_k = top_k
+    c.moe_dim = moe_dim
+    c.num_sink = num_sink
+    c.router = ROUTERS[router]
+    c.logits_dtype = DTYPES[logits_dtype]
+    c.logits_row_stride = num_experts + num_sink if logits_row_stride is None else logits_row_stride
+    c.route_scale = route_scale
+    c.gate_up_format = FORMATS[gate_up_format]
+    c.activation = ACTIVATIONS[activation]
+    c.alpha = alpha
+    c.limit = limit
+    c.has_bias = 1 if has_bias else 0
+    return c
+
+
 def make_config(wl, num_tokens: Optional[int] = None, logits_dtype=torch.float32,
                 logits_row_stride: Optional[int] = None) -> MoEConfig:
     """moe_config_t for a workloads.Workload (num_tokens overrides wl's T)."""
-    c = MoEConfig()
-    c.num_tokens = wl.num_tokens if num_tokens is None else num_tokens
-    c.hidden_dim = wl.hidden_dim
-    c.num_experts = wl.num_experts
-    c.top_k = wl.top_k
-    c.moe_dim = wl.moe_dim
-    c.num_sink = wl.num_sink
-    c.router = ROUTERS[wl.router]
-    c.logits_dtype = DTYPES[logits_dtype]
-    c.logits_row_stride = wl.num_experts + wl.num_sink if logits_row_stride is None else logits_row_stride
-    c.route_scale = wl.route_scale
-    c.gate_up_format = FORMATS[wl.gate_up_format]
-    c.activation = ACTIVATIONS[wl.activation]
-    c.alpha = wl.alpha
-    c.limit = wl.limit
-    c.has_bias = 1 if wl.has_bias else 0
-    return c
+    return config(wl.num_tokens if num_tokens is None else num_tokens, wl.hidden_dim, wl.num_experts, wl.top_k,
+                  wl.moe_dim, router=wl.router, num_sink=wl.num_sink, logits_dtype=logits_dtype,
+                  logits_row_stride=logits_row_stride, route_scale=wl.route_scale,
+                  gate_up_format=wl.gate_up_format, activation=wl.activation, alpha=wl.alpha, limit=wl.limit,
+                  has_bias=wl.has_bias)
 
 
 def _p(t) -> Optional[int]:
