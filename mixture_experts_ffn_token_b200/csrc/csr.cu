@@ -42,10 +42,22 @@ __global__ void __launch_bounds__(kCsrThreads) csr_count_kernel(const int32_t* _
   __syncthreads();
   const int64_t base = static_cast<int64_t>(blockIdx.x) * kCsrChunk;
   const int64_t end = min(base + kCsrChunk, static_cast<int64_t>(R));
+  // all of this thread's slots are loaded before the first is counted
+  constexpr int kPerThread = kCsrChunk / kCsrThreads;
+  int ev[kPerThread];
+  uint32_t live = 0;  // bit q: slot q of this thread exists and its token is not masked
+#pragma unroll
+  for (int q = 0; q < kPerThread; ++q) {
+    const int64_t s = base + threadIdx.x + static_cast<int64_t>(q) * kCsrThreads;
+    const bool on = s < end && slot_live(mask, s, k);
+    ev[q] = on ? idx[s] : 0;
+    live |= on ? (1u << q) : 0u;
+  }
   bool bad = false;
-  for (int64_t s = base + threadIdx.x; s < end; s += blockDim.x) {
-    if (!slot_live(mask, s, k)) continue;
-    const int e = idx[s];
+#pragma unroll
+  for (int q = 0; q < kPerThread; ++q) {
+    if (!((live >> q) & 1u)) continue;
+    const int e = ev[q];
     if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
     else bad = true;
   }
@@ -113,10 +125,18 @@ __global__ void __launch_bounds__(kCsrThreads) csr_scatter_kernel(const int32_t*
   const int64_t wbase = static_cast<int64_t>(blockIdx.x) * kCsrChunk + static_cast<int64_t>(warp) * kSlotsPerWarp;
   int* my = wcnt + warp * E;
   const uint32_t lt_mask = (1u << lane) - 1u;
+  // this lane's slots, loaded once for both passes
+  constexpr int kRounds = kSlotsPerWarp / 32;
+  int ev[kRounds];
+#pragma unroll
+  for (int q = 0; q < kRounds; ++q) {
+    const int64_t s = wbase + 32 * q + lane;
+    ev[q] = s < R && slot_live(mask, s, k) ? idx[s] : -1;
+  }
   // pass 1: per-warp histogram
-  for (int r = 0; r < kSlotsPerWarp; r += 32) {
-    const int64_t s = wbase + r + lane;
-    const int e = s < R && slot_live(mask, s, k) ? idx[s] : -1;
+#pragma unroll
+  for (int q = 0; q < kRounds; ++q) {
+    const int e = ev[q];
     const bool ok = e >= 0 && e < E;
     const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : E + lane);
     if (ok && (peers & lt_mask) == 0) my[e] += __popc(peers);
@@ -135,9 +155,10 @@ __global__ void __launch_bounds__(kCsrThreads) csr_scatter_kernel(const int32_t*
   __syncthreads();
   // pass 2: positions in slot order
   const int32_t* cb = chunk_base + static_cast<int64_t>(blockIdx.x) * E;
-  for (int r = 0; r < kSlotsPerWarp; r += 32) {
-    const int64_t s = wbase + r + lane;
-    const int e = s < R && slot_live(mask, s, k) ? idx[s] : -1;
+#pragma unroll
+  for (int q = 0; q < kRounds; ++q) {
+    const int64_t s = wbase + 32 * q + lane;
+    const int e = ev[q];
     const bool ok = e >= 0 && e < E;
     const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : E + lane);
     int base = 0;
