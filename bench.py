@@ -279,9 +279,9 @@ def run_reference(args, wl):
     return 0
 
 
-def config_block(wl, world):
+def config_block(wl, world, graph=False):
     big = 3 * wl.num_experts * wl.hidden_dim * wl.moe_dim * 2
-    return {"workload": wl.name, "num_tokens": wl.num_tokens, "hidden_dim": wl.hidden_dim,
+    return {"workload": wl.name, "launch": "cuda_graph" if graph else "eager", "num_tokens": wl.num_tokens, "hidden_dim": wl.hidden_dim,
             "num_experts": wl.num_experts, "top_k": wl.top_k, "moe_dim": wl.moe_dim, "num_sink": wl.num_sink,
             "router": wl.router, "gate_up_format": wl.gate_up_format, "activation": wl.activation,
             "has_bias": wl.has_bias, "parallelism": f"replicas x{world}",
@@ -431,12 +431,25 @@ def run_gpu(args, wl):
 
     # ---------------- timed region: K steps of moe_forward between two CUDA
     # events on the launching stream (max over ranks); L2 flushed between
-    # steps when the inputs would fit in it
+    # steps when the inputs would fit in it.  With --graph (default) one step
+    # is captured in a CUDA graph and each timed step replays it, which takes
+    # the host's launch work off the timeline; the layer itself is the same.
+    timed = step
+    graph = None
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        graph.replay()
+        torch.cuda.synchronize()
+        if abi.moe_device_status(ws) != 0:
+            raise RuntimeError("device status set by the captured step")
+        timed = graph.replay
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        elapsed_ms = timed_steps(step, args.steps, stream, flush)
+        elapsed_ms = timed_steps(timed, args.steps, stream, flush)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -526,7 +539,7 @@ def run_gpu(args, wl):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random-init expert weights N(0,0.02))",
-        "config": config_block(wl, world),
+        "config": config_block(wl, world, graph=args.graph),
         "tflops": flops / (ms_per_step / 1e3) / 1e12,
         "weight_gbs": (wbytes + workload_bytes(wl)) / (ms_per_step / 1e3) / 1e9,
         "experts_touched": used,
@@ -538,6 +551,7 @@ def run_gpu(args, wl):
         "single_launch_ffn": fused,
         "clocks": clock_summary,
     }
+    del graph
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, inp)
     if rank == 0:
@@ -563,6 +577,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
+                    help="time replays of a CUDA graph of one step (default) or eager calls")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -377,3 +377,32 @@ def test_nvtx_ranges_change_nothing():
     env = dict(os.environ, MOE_B200_NVTX="1")
     r = subprocess.run([sys.executable, "-c", script], env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stderr[-2000:]
+
+
+@pytest.mark.parametrize("name", ["sink_small", "gptoss_small", "decode_small"])
+def test_cuda_graph_capture(name):
+    """moe_forward allocates nothing and never synchronizes, so it can be
+    captured in a CUDA graph (cooperative single launch and programmatic
+    dependent launches included); every replay gives the eager result."""
+    wl = SMALL[name]
+    d = to_dev(make_inputs(wl, 16))
+    eager = GpuRun(wl, d)
+    assert eager.status == 0
+    T, H, k, S = wl.num_tokens, wl.hidden_dim, wl.top_k, wl.num_sink
+    ws = torch.empty_like(eager.ws)
+    out = torch.zeros((T, H), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    kw = dict(gate_up_b=d["b_gu"], down_b=d["b_d"], expert_bias=d["expert_bias"], global_scale=d["global_scale"],
+              expert_indices_out=idx)
+    abi.moe_forward(eager.cfg, d["x"], d["logits"], d["W_gu"], d["W_d"], out, ws, **kw)  # warm-up before capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        abi.moe_forward(eager.cfg, d["x"], d["logits"], d["W_gu"], d["W_d"], out, ws, **kw)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert abi.moe_device_status(ws) == 0
+        assert torch.equal(out, eager.out) and torch.equal(idx, eager.idx)
+    del g
