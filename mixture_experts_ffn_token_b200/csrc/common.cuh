@@ -324,10 +324,16 @@ __device__ __forceinline__ float gated_act(int act, float g, float u, float alph
     g = fminf(g, limit);
     u = fminf(fmaxf(u, -limit), limit);
   }
-  if (act == 0) return g / (1.f + expf(-g)) * u;
-  if (act == 1) return g / (1.f + expf(-alpha * g)) * (u + 1.f);
+  // Fast forms: the hardware exp2 and reciprocal approximations behind
+  // __expf / __fdividef, and tanh.approx.f32 (relative error about 2^-11),
+  // all well below the bf16 rounding of the stored h.  For g -> -inf the
+  // exponential overflows and the quotient is 0, as the limit is.
+  if (act == 0) return __fdividef(g, 1.f + __expf(-g)) * u;
+  if (act == 1) return __fdividef(g, 1.f + __expf(-alpha * g)) * (u + 1.f);
   const float inner = 0.7978845608028654f * (g + 0.044715f * g * g * g);
-  return 0.5f * g * (1.f + tanhf(inner)) * u;
+  float th;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(inner));
+  return 0.5f * g * (1.f + th) * u;
 }
 
 }  // namespace moe
