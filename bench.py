@@ -312,10 +312,13 @@ def timed_steps(step, steps, stream, flush):
     return total
 
 
-def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None):
+def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None, copy_streams=1):
     """K steps of moe_forward (moe_forward_ex when `make_ex` builds its extras
     from a device token mask) fed from, and returning to, pinned host memory.
     The token mask, when there is one, is a per-step input and is copied too.
+    Each per-step copy is split by rows over `copy_streams` streams per
+    direction (so that several copy engines share it), double-buffered so
+    that step i's copies overlap the compute of its neighbours.
     Returns the device time (max over ranks) of the whole region in ms."""
     T, H = inp["x"].shape
     x_h = inp["x"].cpu().pin_memory()
@@ -328,41 +331,51 @@ def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None):
     x_d = [torch.empty_like(inp["x"]) for _ in range(2)]
     lg_d = [torch.empty_like(inp["logits"]) for _ in range(2)]
     out_d = [torch.empty((T, H), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
-    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    n = max(1, min(copy_streams, T))
+    h2d = [torch.cuda.Stream() for _ in range(n)]
+    d2h = [torch.cuda.Stream() for _ in range(n)]
+    cut = [T * q // n for q in range(n + 1)]  # row ranges of the split copies
 
     def region(steps):
-        in_ready = [torch.cuda.Event() for _ in range(steps)]
+        in_ready = [[torch.cuda.Event() for _ in range(n)] for _ in range(steps)]
         fwd_done = [torch.cuda.Event() for _ in range(steps)]
-        out_done = [torch.cuda.Event() for _ in range(steps)]
+        out_done = [[torch.cuda.Event() for _ in range(n)] for _ in range(steps)]
         start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         start.record(stream)
-        h2d.wait_event(start)
-        d2h.wait_event(start)
+        for st in h2d + d2h:
+            st.wait_event(start)
         for i in range(steps):
             b = i % 2
-            with torch.cuda.stream(h2d):
-                if i >= 2:
-                    h2d.wait_event(fwd_done[i - 2])        # buffer b no longer read by step i-2
-                x_d[b].copy_(x_h, non_blocking=True)
-                lg_d[b].copy_(lg_h, non_blocking=True)
-                if has_mask:
-                    mask_d[b].copy_(mask_h, non_blocking=True)
-                in_ready[i].record(h2d)
-            stream.wait_event(in_ready[i])
+            for q, st in enumerate(h2d):
+                lo, hi = cut[q], cut[q + 1]
+                with torch.cuda.stream(st):
+                    if i >= 2:
+                        st.wait_event(fwd_done[i - 2])      # buffer b no longer read by step i-2
+                    x_d[b][lo:hi].copy_(x_h[lo:hi], non_blocking=True)
+                    lg_d[b][lo:hi].copy_(lg_h[lo:hi], non_blocking=True)
+                    if has_mask:
+                        mask_d[b][lo:hi].copy_(mask_h[lo:hi], non_blocking=True)
+                    in_ready[i][q].record(st)
+            for ev in in_ready[i]:
+                stream.wait_event(ev)
             if i >= 2:
-                stream.wait_event(out_done[i - 2])         # out_d[b] copied out by step i-2
+                for ev in out_done[i - 2]:
+                    stream.wait_event(ev)                   # out_d[b] copied out by step i-2
             if ex_b[b] is None:
                 abi.moe_forward(cfg, x_d[b], lg_d[b], inp["W_gu"], inp["W_d"], out_d[b], ws, stream=stream, **kw)
             else:
                 abi.moe_forward_ex(cfg, ex_b[b], x_d[b], lg_d[b], inp["W_gu"], inp["W_d"], out_d[b], ws,
                                    stream=stream, **kw)
             fwd_done[i].record(stream)
-            with torch.cuda.stream(d2h):
-                d2h.wait_event(fwd_done[i])
-                out_h[b].copy_(out_d[b], non_blocking=True)
-                out_done[i].record(d2h)
-        stream.wait_event(out_done[steps - 1])
-        stream.wait_event(out_done[steps - 2] if steps > 1 else out_done[steps - 1])
+            for q, st in enumerate(d2h):
+                lo, hi = cut[q], cut[q + 1]
+                with torch.cuda.stream(st):
+                    st.wait_event(fwd_done[i])
+                    out_h[b][lo:hi].copy_(out_d[b][lo:hi], non_blocking=True)
+                    out_done[i][q].record(st)
+        for i in range(max(0, steps - 2), steps):
+            for ev in out_done[i]:
+                stream.wait_event(ev)
         stop.record(stream)
         torch.cuda.synchronize()
         return start.elapsed_time(stop)
@@ -479,7 +492,7 @@ def run_gpu(args, wl):
     # from pinned memory and its output device->host inside the timed region.
     # Copies run on their own streams, double-buffered, so step i's copies
     # overlap the compute of its neighbours.
-    e2e_ms = run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex)
+    e2e_ms = run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex, copy_streams=args.copy_streams)
     e2e_value = job_throughput(world, T, e2e_ms / args.steps)
     x_h_bytes = inp["x"].numel() * 2 + inp["logits"].numel() * 4
     if inp["token_mask"] is not None:
@@ -577,6 +590,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--copy-streams", type=int, default=1,
+                    help="streams per direction that share each e2e step's host<->device copies")
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="time replays of a CUDA graph of one step (default) or eager calls")
     args = ap.parse_args()
