@@ -203,7 +203,10 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* log
  * CSR count, CSR scan, CSR scatter, gather, gate_up GEMM, down GEMM and
  * combine, and after the combine, so a caller can time each kernel on the
  * stream it runs on.  With the single-launch FFN the "gate_up GEMM" stage
- * is the fused launch and the "down GEMM" stage is empty. */
+ * is the fused launch and the "down GEMM" stage is empty.  A NULL entry of
+ * the array is skipped (so a caller can time one stage alone); a NULL array
+ * is MOE_ERR_INVALID_ARGUMENT.  Under stream capture the events become
+ * external event-record nodes, so each replay of the graph records them. */
 /* *enabled = 1 if moe_grouped_ffn / moe_forward / moe_forward_ex called now
  * in this process run the two GEMMs as one launch, 0 if as two (the
  * MOE_B200_SINGLE_LAUNCH setting, read at each call). */
@@ -267,7 +270,7 @@ moe_status_t moe_workspace_size_ex(const moe_config_t* cfg, const moe_extras_t* 
 
 /* moe_forward with the extensions above.  Same arguments and conventions as
  * moe_forward, plus `extras` (NULL = none) and stage_events (NULL, or
- * MOE_NUM_STAGE_EVENTS_EX caller-created cudaEvent_t).  The output is
+ * MOE_NUM_STAGE_EVENTS_EX caller-created cudaEvent_t, NULL entries skipped).  The output is
  *   out[t] = mask[t] * ( sum_j  w_tj * FFN_e(tj)(x_t)          (or FFN(w_tj x_t))
  *                      + sum_i  g_ti * SharedFFN_i(x_t) )      (or SharedFFN_i(g_ti x_t))
  * summed in fp32 (routed slots j ascending, then shared i ascending). */

@@ -237,16 +237,27 @@ def moe_forward(cfg, x, logits, gate_up_w, down_w, out, workspace, gate_up_b=Non
                                       _p(workspace), workspace.numel(), _stream(stream)), "moe_forward")
 
 
+def _event_handles(events, stream):
+    """cudaEvent_t handles of torch.cuda.Event objects (None stays NULL)."""
+    handles = []
+    for ev in events:
+        if ev is None:
+            handles.append(None)
+            continue
+        if ev.cuda_event == 0:      # torch creates the CUDA event on its first record
+            ev.record(stream)
+        handles.append(ev.cuda_event)
+    return handles
+
+
 def moe_forward_timed(cfg, events, x, logits, gate_up_w, down_w, out, workspace, gate_up_b=None, down_b=None,
                       expert_bias=None, global_scale=None, expert_indices_out=None, expert_weights_out=None,
                       sink_weights_out=None, stream=None):
-    """moe_forward recording torch.cuda.Event objects `events` (9) between stages."""
+    """moe_forward recording torch.cuda.Event objects `events` (9, None
+    entries skipped) between stages."""
     if len(events) != NUM_STAGE_EVENTS:
         raise ValueError(f"moe_forward_timed needs {NUM_STAGE_EVENTS} events")
-    for ev in events:
-        if ev.cuda_event == 0:      # torch creates the CUDA event on its first record
-            ev.record(stream)
-    arr = (ctypes.c_void_p * NUM_STAGE_EVENTS)(*[ev.cuda_event for ev in events])
+    arr = (ctypes.c_void_p * NUM_STAGE_EVENTS)(*_event_handles(events, stream))
     _check(load_library().moe_forward_timed(ctypes.byref(cfg), _p(x), _p(logits), _p(expert_bias),
                                             _p(global_scale), _p(gate_up_w), _p(gate_up_b), _p(down_w), _p(down_b),
                                             _p(out), _p(expert_indices_out), _p(expert_weights_out),
@@ -278,10 +289,7 @@ def moe_forward_ex(cfg, extras, x, logits, gate_up_w, down_w, out, workspace, ga
     if events is not None:
         if len(events) != NUM_STAGE_EVENTS_EX:
             raise ValueError(f"moe_forward_ex needs {NUM_STAGE_EVENTS_EX} events")
-        for ev in events:
-            if ev.cuda_event == 0:
-                ev.record(stream)
-        arr = (ctypes.c_void_p * NUM_STAGE_EVENTS_EX)(*[ev.cuda_event for ev in events])
+        arr = (ctypes.c_void_p * NUM_STAGE_EVENTS_EX)(*_event_handles(events, stream))
     ex = None if extras is None else ctypes.byref(extras)
     _check(load_library().moe_forward_ex(ctypes.byref(cfg), ex, _p(x), _p(logits), _p(expert_bias),
                                          _p(global_scale), _p(gate_up_w), _p(gate_up_b), _p(down_w), _p(down_b),

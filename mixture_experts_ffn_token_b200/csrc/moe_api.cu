@@ -232,7 +232,15 @@ struct Recorder {
   cudaEvent_t const* ev;
   cudaStream_t stream;
   void operator()(int i) const {
-    if (ev != nullptr) cudaEventRecord(ev[i], stream);
+    if (ev == nullptr || ev[i] == nullptr) return;  // NULL slots are skipped
+    // Under stream capture an event is recorded as an external event-record
+    // node, so every replay of the graph records it (a plain record would
+    // only become a dependency edge of the capture).
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+      cudaEventRecordWithFlags(ev[i], stream, cudaEventRecordExternal);
+    else
+      cudaEventRecord(ev[i], stream);
   }
 };
 
@@ -591,8 +599,6 @@ moe_status_t moe_forward_timed(const moe_config_t* cfg, const void* x, const voi
                                float* expert_weights_out, float* sink_weights_out, void* workspace,
                                size_t workspace_bytes, moe_stream_t stream, void* const* stage_events) {
   if (stage_events == nullptr) return MOE_ERR_INVALID_ARGUMENT;
-  for (int i = 0; i < MOE_NUM_STAGE_EVENTS; ++i)
-    if (stage_events[i] == nullptr) return MOE_ERR_INVALID_ARGUMENT;
   return forward_impl(cfg, nullptr, x, logits, expert_bias, global_scale, gate_up_w, gate_up_b, down_w, down_b, out,
                       expert_indices_out, expert_weights_out, sink_weights_out, workspace, workspace_bytes,
                       reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<cudaEvent_t const*>(stage_events));
@@ -613,9 +619,6 @@ moe_status_t moe_forward_ex(const moe_config_t* cfg, const moe_extras_t* extras,
                             const void* gate_up_b, const void* down_w, const void* down_b, void* out,
                             int32_t* expert_indices_out, float* expert_weights_out, float* sink_weights_out,
                             void* workspace, size_t workspace_bytes, moe_stream_t stream, void* const* stage_events) {
-  if (stage_events != nullptr)
-    for (int i = 0; i < MOE_NUM_STAGE_EVENTS_EX; ++i)
-      if (stage_events[i] == nullptr) return MOE_ERR_INVALID_ARGUMENT;
   moe_extras_t none;
   std::memset(&none, 0, sizeof(none));
   return forward_impl(cfg, extras != nullptr ? extras : &none, x, logits, expert_bias, global_scale, gate_up_w,

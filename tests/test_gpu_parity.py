@@ -406,3 +406,36 @@ def test_cuda_graph_capture(name):
         assert abi.moe_device_status(ws) == 0
         assert torch.equal(out, eager.out) and torch.equal(idx, eager.idx)
     del g
+
+
+def test_stage_events_inside_a_cuda_graph():
+    """moe_forward_timed with only the GEMM stage's pair of events set (the
+    other slots NULL), captured in a CUDA graph: every replay records that
+    pair, and the stage time is positive and shorter than the whole step."""
+    wl = SMALL["sink_small"]
+    d = to_dev(make_inputs(wl, 17))
+    eager = GpuRun(wl, d)
+    ws = torch.empty_like(eager.ws)
+    out = torch.empty_like(eager.out)
+    kw = dict(expert_bias=d["expert_bias"], global_scale=d["global_scale"])
+    a, b = torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True)
+    s0, s1 = torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True)
+    evs = [None] * abi.NUM_STAGE_EVENTS
+    evs[5], evs[6] = a, b                       # around the gate_up stage (the single launch by default)
+    for ev in (a, b, s0, s1):
+        ev.record()
+    abi.moe_forward_timed(eager.cfg, evs, d["x"], d["logits"], d["W_gu"], d["W_d"], out, ws, **kw)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        s0.record()
+        abi.moe_forward_timed(eager.cfg, evs, d["x"], d["logits"], d["W_gu"], d["W_d"], out, ws, **kw)
+        s1.record()
+    for _ in range(2):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        stage, whole = a.elapsed_time(b), s0.elapsed_time(s1)
+        assert 0.0 < stage < whole, (stage, whole)
+        assert torch.equal(out, eager.out)
+    del g
