@@ -439,3 +439,34 @@ def test_stage_events_inside_a_cuda_graph():
         assert 0.0 < stage < whole, (stage, whole)
         assert torch.equal(out, eager.out)
     del g
+
+
+@pytest.mark.parametrize("name", ["sink_small", "gptoss_small", "decode_small", "mixtral_small"])
+@pytest.mark.parametrize("single_launch", ["1", "0"])
+def test_no_writes_past_any_buffer(name, single_launch, monkeypatch):
+    """Canaries after the workspace and after every routing output: the
+    kernels write only inside the sizes the API states."""
+    monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", single_launch)
+    wl = SMALL[name]
+    d = to_dev(make_inputs(wl, 18))
+    cfg = abi.make_config(wl)
+    T, H, k, S = wl.num_tokens, wl.hidden_dim, wl.top_k, wl.num_sink
+    guard = 4096
+    need = abi.moe_workspace_size(cfg)
+    ws_full = torch.full((need + guard,), 0xA5, dtype=torch.uint8, device="cuda")
+    ws = ws_full[:need]
+    idx_full = torch.full((T * k + guard,), -12345, dtype=torch.int32, device="cuda")
+    w_full = torch.full((T * k + guard,), -3.0, dtype=torch.float32, device="cuda")
+    sink_full = torch.full((T * S + guard,), -5.0, dtype=torch.float32, device="cuda")
+    out_full = torch.full((T * H + guard,), -7.0, dtype=torch.bfloat16, device="cuda")
+    abi.moe_forward(cfg, d["x"], d["logits"], d["W_gu"], d["W_d"], out_full[:T * H].view(T, H), ws,
+                    gate_up_b=d["b_gu"], down_b=d["b_d"], expert_bias=d["expert_bias"],
+                    global_scale=d["global_scale"], expert_indices_out=idx_full[:T * k].view(T, k),
+                    expert_weights_out=w_full[:T * k].view(T, k),
+                    sink_weights_out=sink_full[:T * S].view(T, S) if S > 0 else None)
+    torch.cuda.synchronize()
+    assert abi.moe_device_status(ws) == 0
+    assert (ws_full[need:] == 0xA5).all(), "workspace guard overwritten"
+    assert (idx_full[T * k:] == -12345).all() and (w_full[T * k:] == -3.0).all()
+    assert (sink_full[T * S:] == -5.0).all()
+    assert (out_full[T * H:] == -7.0).all()
