@@ -758,8 +758,12 @@ constexpr size_t smem_bytes_for(int E) {
 // Clusters of two that can be resident at once (cached per kernel).
 template <int MODE>
 int max_pair_clusters(size_t smem, int num_sms) {
-  static int cached = 0;
-  if (cached > 0) return cached;
+  // occupancy depends on the device: cached per device
+  constexpr int kDevices = 64;
+  static int cached[kDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) return num_sms / 2;
+  if (cached[dev] > 0) return cached[dev];
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -774,7 +778,7 @@ int max_pair_clusters(size_t smem, int num_sms) {
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<MODE, 2, false>, &cfg) != cudaSuccess || n <= 0)
     n = num_sms / 2;
-  cached = n;
+  cached[dev] = n;
   return n;
 }
 

@@ -249,8 +249,12 @@ cudaError_t launch_small_npl(const RouterArgs& a, int32_t* offsets, int32_t* per
   const dim3 block(32 * kSmallWarps);
   const dim3 one(1);
   // the per-warp histograms need up to (2048 + 32 * 512) * 4 bytes, above the default 48 KB
-  static bool opted_in = false;
-  if (!opted_in) {
+  // function attributes are per device: opt in once for each device
+  constexpr int kDevices = 64;
+  static bool opted_in[kDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) return cudaErrorInvalidDevice;
+  if (!opted_in[dev]) {
     const int max_smem = static_cast<int>((kSmallSlots + static_cast<size_t>(kSmallWarps) * kSmallExperts) * sizeof(int));
     cudaError_t e =
         cudaFuncSetAttribute(route_csr_small_kernel<NPL, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
@@ -264,7 +268,7 @@ cudaError_t launch_small_npl(const RouterArgs& a, int32_t* offsets, int32_t* per
       e = cudaFuncSetAttribute(route_csr_small_kernel<NPL, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                max_smem);
     if (e != cudaSuccess) return e;
-    opted_in = true;
+    opted_in[dev] = true;
   }
   if (a.sink) {
     if (a.logits_bf16)
