@@ -61,10 +61,10 @@ def test_no_extras_equals_forward():
     assert sum(events[i].elapsed_time(events[i + 1]) for i in range(abi.NUM_STAGE_EVENTS_EX - 1)) > 0
 
 
-@pytest.mark.parametrize("name", ["sink_shared", "mixtral_wfirst"])
+@pytest.mark.parametrize("name", ["sink_shared", "mixtral_wfirst", "sink_masked", "mixtral_masked"])
 def test_extension_workloads_full_size_sampled(name):
     import numpy as np
-    wl = WORKLOADS[name]
+    wl = WORKLOADS[name] if name in WORKLOADS else WORKLOADS[name.split("_")[0]].replace(mask_frac=0.3)
     rng = np.random.default_rng(7)
     sample = np.unique(np.concatenate([[0, wl.num_tokens - 1], rng.choice(wl.num_tokens, 10, replace=False)]))
     run_and_check_ex(wl, seed=0, device_inputs=True, sample_tokens=sample)
