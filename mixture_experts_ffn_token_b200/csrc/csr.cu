@@ -296,9 +296,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
 // order, offsets[i] = i*T, and row i*T + t is slot t*Ns + i of the [T, Ns]
 // slot space (so slot / Ns is the token and the gates are indexed by slot).
 __global__ void __launch_bounds__(256) shared_index_kernel(int T, int Ns, int32_t* __restrict__ offsets,
-                                                           int32_t* __restrict__ perm) {
+                                                           int32_t* __restrict__ perm, int* __restrict__ zero,
+                                                           int n_zero) {
   griddep_wait();  // the previous kernel's results are complete and visible
   griddep_launch_dependents();
+  // clear the shared pass's counters when it has no gather to do it
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_zero; i += gridDim.x * blockDim.x) zero[i] = 0;
   const int64_t n = static_cast<int64_t>(T) * Ns;
   for (int64_t p = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; p < n;
        p += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -310,10 +313,11 @@ __global__ void __launch_bounds__(256) shared_index_kernel(int T, int Ns, int32_
 
 }  // namespace
 
-cudaError_t launch_shared_index(int T, int Ns, int32_t* offsets, int32_t* perm, int num_sms, cudaStream_t stream) {
+cudaError_t launch_shared_index(int T, int Ns, int32_t* offsets, int32_t* perm, int num_sms, cudaStream_t stream,
+                                int* zero, int n_zero) {
   const int64_t n = static_cast<int64_t>(T) * Ns;
   const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, num_sms * 4)));
-  return launch_pdl(shared_index_kernel, dim3(blocks), dim3(256), 0, stream, T, Ns, offsets, perm);
+  return launch_pdl(shared_index_kernel, dim3(blocks), dim3(256), 0, stream, T, Ns, offsets, perm, zero, n_zero);
 }
 
 cudaError_t launch_csr_count(const int32_t* idx, int R, int E, int32_t* chunk_counts, int* status,

@@ -102,6 +102,7 @@ struct GemmParams {
   // of that wait
   int extra_arrivals;
   unsigned long long dep_timeout_ns;
+  int a_direct;  // gate_up: A rows are rows within the expert's segment (A = x)
 };
 
 struct TileCoord {
@@ -494,7 +495,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool ph2 = FUSED && t >= total1;
         const TileCoord tc = ph2 ? decode_tile(t - total1, p2.n_tiles, p.E, s_mt, s_off, G::PIECE)
                                  : decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
-        const int arow = tc.row0 + static_cast<int>(rank) * BM;
+        const int arow = (!ph2 && p.a_direct ? tc.row0 - s_off[tc.e] : tc.row0) + static_cast<int>(rank) * BM;
         const int nkb = ph2 ? p2.num_kb : p.num_kb;
         if constexpr (FUSED) {
           if (ph2) {
@@ -875,7 +876,9 @@ cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& ma
   const bool down = MODE == MODE_DOWN;
   const int K = down ? a.D : a.H;
   {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(a.R)};
+    // with a_direct the A operand is x: T rows, indexed by the row within an expert
+    const cuuint64_t rows = static_cast<cuuint64_t>(!down && a.a_direct ? a.T : a.R);
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), rows};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
     const cuuint32_t box[2] = {64, BM};
     if (!encode_bf16_map(&mapA, a.A, 2, dims, strides, box)) return cudaErrorInvalidValue;
@@ -914,6 +917,7 @@ cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& ma
     if (!encode_bf16_map(&mapB, a.W, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
   p.offsets = a.offsets;
+  p.a_direct = !down && a.a_direct ? 1 : 0;
   p.perm = a.perm;
   p.weights = a.weights;
   p.bias = a.bias;

@@ -65,7 +65,10 @@ cudaError_t launch_csr_scan(const int32_t* chunk_counts, int nchunks, int E, int
                             int32_t* offsets, cudaStream_t stream);
 cudaError_t launch_csr_scatter(const int32_t* idx, int R, int E, const int32_t* chunk_base, int32_t* perm,
                                int32_t* inv, const uint8_t* mask, int k, cudaStream_t stream);
-cudaError_t launch_shared_index(int T, int Ns, int32_t* offsets, int32_t* perm, int num_sms, cudaStream_t stream);
+// shared slots: offsets[i] = i*T, perm[i*T + t] = t*Ns + i; also clears
+// zero[0 .. n_zero) (may be null / 0).
+cudaError_t launch_shared_index(int T, int Ns, int32_t* offsets, int32_t* perm, int num_sms, cudaStream_t stream,
+                                int* zero = nullptr, int n_zero = 0);
 
 // ----------------------------------------------------- gather and combine
 // scale (may be null): per-slot factor applied to the gathered row.
@@ -92,6 +95,9 @@ struct GroupedGemmArgs {
   float alpha, limit;
   // operands (device)
   const __nv_bfloat16* A;   // Xp [R,H] (gate_up) or h [R,D] (down)
+  // gate_up only: A is x [T,H] itself and a slot's A row is its row within
+  // its expert's segment (the shared experts' slots, token order per expert)
+  int a_direct = 0;
   const __nv_bfloat16* W;   // [E,H,2D] (gate_up) or [E,D,H] (down)
   const __nv_bfloat16* bias;// [E,2D] / [E,H] or null
   __nv_bfloat16* out;       // h [R,D] (gate_up) or Y [R,H] slot rows (down)

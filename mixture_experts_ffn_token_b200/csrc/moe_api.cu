@@ -250,17 +250,20 @@ struct Recorder {
 // overwrites Xp (the gate_up GEMM is done with it); the single launch
 // writes Y to y_sep and counts arrivals in arr.  *y_out = where Y is.
 // rec(base..base+2) before each stage (the down stage is empty when fused).
+// a_direct: the gate_up GEMM reads x itself (a slot's A row is its row within
+// its expert's segment, as for the shared experts' slots); no gather runs, so
+// the caller has cleared arr.
 moe_status_t enqueue_grouped_pass(const moe_config_t* c, int E, int k, int D, const void* x, const void* gate_up_w,
                                   const void* gate_up_b, const void* down_w, const void* down_b,
                                   const int32_t* offsets, const int32_t* perm, const float* scale,
                                   const float* weights, __nv_bfloat16* xp, __nv_bfloat16* h, __nv_bfloat16* y_sep,
                                   int* arr, __nv_bfloat16** y_out, int* status, int num_sms, cudaStream_t stream,
-                                  const Recorder& rec, int base) {
+                                  const Recorder& rec, int base, bool a_direct = false) {
   const int T = c->num_tokens, H = c->hidden_dim;
   const int R = T * k;
   const bool fused = single_launch();
   rec(base);
-  {
+  if (!a_direct) {
     const NvtxRange range("moe.gather");
     if (moe::launch_gather(static_cast<const __nv_bfloat16*>(x), perm, offsets, E, R, k, H, scale, xp, status,
                            num_sms, stream, fused ? arr : nullptr, fused ? moe::mega_ffn_counters(R, E) : 0) !=
@@ -283,7 +286,8 @@ moe_status_t enqueue_grouped_pass(const moe_config_t* c, int E, int k, int D, co
   g.limit = c->limit;
   g.status = status;
   g.num_sms = num_sms;
-  g.A = xp;
+  g.A = a_direct ? static_cast<const __nv_bfloat16*>(x) : xp;
+  g.a_direct = a_direct ? 1 : 0;
   g.W = static_cast<const __nv_bfloat16*>(gate_up_w);
   g.bias = static_cast<const __nv_bfloat16*>(gate_up_b);
   g.out = h;
@@ -471,16 +475,23 @@ moe_status_t forward_impl(const moe_config_t* cfg, const moe_extras_t* extras, c
     // weights (sink router) or by 1
     int32_t* s_off = at<int32_t>(ws, L.sh_offsets);
     int32_t* s_perm = at<int32_t>(ws, L.sh_perm);
+    // Shared expert i's slots are the tokens in order, so unless the gate
+    // scales the input its gate_up GEMM reads x directly and no gather runs;
+    // the index kernel then clears the pass's counters.
+    const bool direct = !ex.weight_first;
+    const int64_t Rs = static_cast<int64_t>(T) * ex.Ns;
     {
       const NvtxRange range("moe.shared_index");
-      if (moe::launch_shared_index(T, ex.Ns, s_off, s_perm, num_sms, stream) != cudaSuccess) return MOE_ERR_CUDA;
+      if (moe::launch_shared_index(T, ex.Ns, s_off, s_perm, num_sms, stream, direct ? at<int>(ws, L.sh_arr) : nullptr,
+                                   direct ? moe::mega_ffn_counters(static_cast<int>(Rs), ex.Ns) : 0) != cudaSuccess)
+        return MOE_ERR_CUDA;
     }
     const float* gates = cfg->router == MOE_ROUTER_SIGMOID_SINK ? sink : nullptr;
     st = enqueue_grouped_pass(cfg, ex.Ns, ex.Ns, ex.Ds, x, ex.s_gu_w, ex.s_gu_b, ex.s_d_w, ex.s_d_b, s_off, s_perm,
                               ex.weight_first ? gates : nullptr, ex.weight_first ? nullptr : gates,
                               at<__nv_bfloat16>(ws, L.sh_x), at<__nv_bfloat16>(ws, L.sh_h),
                               at<__nv_bfloat16>(ws, L.sh_y), at<int>(ws, L.sh_arr), &ys, status, num_sms, stream,
-                              rec, 8);
+                              rec, 8, direct);
     if (st != MOE_OK) return st;
   } else {
     for (int i = 8; i <= 10; ++i) rec(i);
