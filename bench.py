@@ -120,6 +120,10 @@ class ClockSampler:
             uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
             self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            try:  # read only, to tell a lowered power limit from the usual one
+                self.limit_w = pynvml.nvmlDeviceGetEnforcedPowerLimit(self.handle) / 1000.0
+            except Exception:
+                self.limit_w = None
             self.nvml = pynvml
         except Exception as exc:  # no NVML: report it instead of guessing
             self.error = f"nvml unavailable: {exc}"
@@ -157,7 +161,10 @@ class ClockSampler:
                           if mask & getattr(p, attr)})
         return {"sm_mhz": statistics.median(s[0] for s in self.samples), "sm_max_mhz": self.max_mhz,
                 "reasons": reasons, "samples": len(self.samples), "source": "nvml",
-                "power_w_max": max(s[2] for s in self.samples)}
+                # NVML's power reading is averaged over about a second, so
+                # over a short timed region it stays below the limit even
+                # while sw_power_cap is active
+                "power_w_max": max(s[2] for s in self.samples), "power_limit_w": self.limit_w}
 
 
 def kernel_traffic(workload, kernel):
