@@ -20,6 +20,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import time
@@ -181,11 +182,29 @@ def kernel_traffic(workload, kernel):
     src = os.path.join(ROOT, ent.get("source", ""))
     if not os.path.isfile(src):
         return None
-    with open(src, "rb") as f:
-        digest = hashlib.sha256(f.read()).hexdigest()[:16]
-    if ent.get("source_sha256_16") != digest:
+    if ent.get("code_sha256_16") != code_digest(src):
         return None
     return ent.get("bytes_per_launch")
+
+
+_C_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'|//[^\n]*|/\*.*?\*/|\s+', re.S)
+
+
+def code_digest(path):
+    """sha256[:16] of a C/C++/CUDA source with its comments and whitespace
+    removed (string and character literals kept): it changes when the code
+    changes, not when a comment does."""
+    with open(path, encoding="utf-8") as f:
+        text = f.read()
+
+    def keep(m):
+        tok = m.group(0)
+        if tok.startswith(("//", "/*")) or tok.isspace():
+            return " "
+        return tok
+
+    code = " ".join(_C_TOKENS.sub(keep, text).split())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 # ---------------------------------------------------------------- oracle arm

@@ -12,29 +12,42 @@
 //
 // Kernel design (one persistent CTA per SM, 320 threads):
 //   warp 0      TMA producer: for every tile and 64-wide K block, one 128x64
-//               box of A (K-major, 128-byte swizzle) and four 64x64 boxes of
-//               B (N-major, 128-byte swizzle) into a 4-stage ring, completion
-//               on a full[stage] mbarrier;
+//               box of A (K-major, 128-byte swizzle) and the 64x256 B tile
+//               (N-major, 128-byte swizzle) into a 4-stage ring of 48 KB
+//               stages, completion on a full[stage] mbarrier.  B arrives in
+//               one copy through a {64 columns, K, column block, (gate/up,)
+//               E} view of the weights where the column count is a multiple
+//               of 64, else as four 64-column boxes (same shared image);
 //   warp 1      TMEM allocator and MMA issuer: one thread issues four
 //               tcgen05.mma 128x256x16 per stage (bf16 in, fp32 accumulate in
-//               TMEM) and tcgen05.commit's the stage back to the producer;
-//               two 256-column accumulators alternate between tiles;
-//   warps 2..9  epilogue: tcgen05.ld of their 32 TMEM lanes (one output row
-//               per thread; two warps per lane quadrant split the columns),
-//               bias + activation (gate_up) or bias x weight (down) in fp32,
-//               bf16 stores.
+//               TMEM; M = 64 for a piece of at most 64 rows) and
+//               tcgen05.commit's the stage back to the producer; two
+//               256-column accumulators alternate between tiles;
+//   warps 2..9  epilogue: tcgen05.ld of their 32 TMEM lanes (two warps per
+//               lane quadrant split the columns), bias + activation (gate_up)
+//               or bias x weight (down) in fp32, bf16 stores transposed
+//               through a small shared staging block per warp.
 // Tiles are the ragged expert segments cut in 128-row pieces times the
-// output columns; the per-expert piece counts are rebuilt from the CSR
-// offsets in shared memory at kernel start, and CTAs walk the tile list with
-// a static stride (expert-major, then output column block, then row piece,
-// so CTAs running together share a weight column block through L2).
-// Rows of a piece beyond its expert's segment are computed and discarded.
+// output column blocks; the per-expert piece counts are rebuilt from the CSR
+// offsets in shared memory at kernel start.  Within an expert the order is
+// column block, then row piece, so CTAs running together share a weight
+// column block through L2.  Rows of a piece beyond its expert's segment are
+// computed and discarded.
+//
+// By default both contractions run in ONE cooperative launch (FUSED): the
+// tile list is every gate_up tile, then every down tile; a down tile of a
+// piece starts once all gate_up tiles of that piece have published their h
+// (per-piece arrival counters, release/acquire).  CTAs take tiles with a
+// static stride or, below 256 rows per expert, from an atomic counter.  A
+// variant on CTA pairs (tcgen05 cta_group::2, 256x256 tiles, two launches)
+// is kept selectable.
+//
 // Weights are read in their stored [K, N] (N-contiguous) layout: the B
 // operand is MN-major, which tcgen05 supports for 16-bit types, so no
-// transposed copy of the weights is needed.  Every mbarrier wait is bounded
-// (mbar_wait); a timeout raises a CTA-wide abort, drains the copies and
-// MMAs in flight, frees TMEM and records MOE_DEVICE_ERR_TIMEOUT_* in the
-// status word.
+// transposed copy of the weights is needed.  Every mbarrier wait and
+// cross-CTA wait is bounded; a timeout raises a CTA-wide abort, drains the
+// copies and MMAs in flight, frees TMEM and records MOE_DEVICE_ERR_TIMEOUT_*
+// in the status word.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
