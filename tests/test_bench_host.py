@@ -1,0 +1,55 @@
+"""bench.py's host-side bookkeeping on CPU: the code digest that keys the
+committed DRAM-traffic figures, and the lookup that uses it."""
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+SRC = """// a kernel
+#include "x.h"
+/* block
+   comment */ __global__ void k(int* p) {
+  const char* s = "not // a comment /* either */";
+  p[0] = '/';   // trailing
+}
+"""
+
+
+def _write(tmp_path, name, text):
+    path = tmp_path / name
+    path.write_text(text)
+    return str(path)
+
+
+def test_comments_and_whitespace_do_not_change_the_digest(tmp_path):
+    a = bench.code_digest(_write(tmp_path, "a.cu", SRC))
+    edited = SRC.replace("// a kernel", "// the same kernel, described again\n// over two lines")
+    edited = edited.replace("/* block\n   comment */", "/* another */").replace("  p[0]", "\tp[0]")
+    assert bench.code_digest(_write(tmp_path, "b.cu", edited)) == a
+
+
+def test_code_and_string_literals_change_the_digest(tmp_path):
+    a = bench.code_digest(_write(tmp_path, "a.cu", SRC))
+    assert bench.code_digest(_write(tmp_path, "b.cu", SRC.replace("p[0] =", "p[1] ="))) != a
+    # a "//" inside a string literal is code, not a comment
+    assert bench.code_digest(_write(tmp_path, "c.cu", SRC.replace("not // a", "not // b"))) != a
+    assert bench.code_digest(_write(tmp_path, "d.cu", SRC.replace("'/'", "'*'"))) != a
+
+
+def test_traffic_figures_are_used_only_for_the_captured_code():
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        table = json.load(f)
+    for workload, kernels in table.items():
+        if workload.startswith("_"):
+            continue
+        for kernel, ent in kernels.items():
+            src = os.path.join(ROOT, ent["source"])
+            current = bench.code_digest(src) == ent["code_sha256_16"]
+            got = bench.kernel_traffic(workload, kernel)
+            assert got == (ent["bytes_per_launch"] if current else None)
+            assert ent["bytes_per_launch"] == ent["read"] + ent["write"]
+    assert bench.kernel_traffic("no_such_workload", "mega_ffn") is None
