@@ -91,6 +91,7 @@ struct Geo {
 // row r in TMEM lane 32*(r/16) + r%16: the first 16 lanes of each 32-lane
 // quadrant, so epilogue warp q reads rows 16q .. 16q+15 from its own lanes.
 constexpr int HALF_ROWS = 64;
+constexpr int HALF_A_BYTES = HALF_ROWS * BK * 2;  // 8 KB: the A rows a half tile copies
 constexpr uint32_t IDESC_HALF = idesc_bf16_f32(HALF_ROWS, BN, /*a_mn_major=*/false, /*b_mn_major=*/true);
 
 constexpr int MODE_GATE_UP_CONCAT = 0;
@@ -366,6 +367,7 @@ template <int MODE, int PAIR, bool FUSED>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                         const __grid_constant__ CUtensorMap mapA2, const __grid_constant__ CUtensorMap mapB2,
+                        const __grid_constant__ CUtensorMap mapAh, const __grid_constant__ CUtensorMap mapA2h,
                         const GemmParams p, const GemmParams p2, int* arrivals, int* sched) {
   static_assert(!FUSED || (PAIR == 1 && MODE != MODE_DOWN), "the fused form is gate_up then down, one CTA a tile");
   using G = Geo<PAIR>;
@@ -510,6 +512,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                  : decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
         const int arow = (!ph2 && p.a_direct ? tc.row0 - s_off[tc.e] : tc.row0) + static_cast<int>(rank) * BM;
         const int nkb = ph2 ? p2.num_kb : p.num_kb;
+        // a half tile (at most 64 rows, M = 64 MMAs) copies only 64 rows of A
+        const bool half = PAIR == 1 && tc.rows <= HALF_ROWS;
+        const uint32_t stage_tx = half ? G::STAGE_BYTES - HALF_A_BYTES : G::STAGE_BYTES;
         if constexpr (FUSED) {
           if (ph2) {
             if (!wait_arrivals(arrivals + tc.piece, arrivals_needed, abort_flag, p.status, p.err_bit,
@@ -534,8 +539,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int kc = kb * BK;
           if (FUSED && ph2) {
             // down tile: h rows of the piece, 256 columns of W_d
-            mbar_arrive_expect_tx(fb, G::STAGE_BYTES);
-            tma_load_2d(sa, &mapA2, fb, kc, arow);
+            mbar_arrive_expect_tx(fb, stage_tx);
+            tma_load_2d(sa, half ? &mapA2h : &mapA2, fb, kc, arow);
             if (p2.b_one_box) {
               tma_load_4d(sb, &mapB2, fb, 0, kc, 4 * tc.n, tc.e);
             } else {
@@ -546,13 +551,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           } else if (PAIR == 1 && p.b_one_box) {
             // {64 columns, K, column block, (gate/up,) E} view: one copy lays
             // the four 64-column boxes out exactly as four copies would
-            mbar_arrive_expect_tx(fb, G::STAGE_BYTES);
-            tma_load_2d(sa, &mapA, fb, kc, arow);
+            mbar_arrive_expect_tx(fb, stage_tx);
+            tma_load_2d(sa, half ? &mapAh : &mapA, fb, kc, arow);
             if constexpr (MODE == MODE_GATE_UP_CONCAT) tma_load_5d(sb, &mapB, fb, 0, kc, 2 * tc.n, 0, tc.e);
             else tma_load_4d(sb, &mapB, fb, 0, kc, 4 * tc.n, tc.e);
           } else if constexpr (PAIR == 1) {
-            mbar_arrive_expect_tx(fb, G::STAGE_BYTES);
-            tma_load_2d(sa, &mapA, fb, kc, arow);
+            mbar_arrive_expect_tx(fb, stage_tx);
+            tma_load_2d(sa, half ? &mapAh : &mapA, fb, kc, arow);
             if constexpr (MODE == MODE_GATE_UP_CONCAT) {
               // 4-D view {D, 2 (gate/up), H, E}: two gate boxes then two up boxes.
               const int c0 = tc.n * 128;
@@ -816,8 +821,8 @@ int choose_pair(int /*R*/, int /*E*/) {
 }
 
 template <int MODE, int PAIR>
-cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmParams& p, int num_sms,
-                        cudaStream_t stream) {
+cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const CUtensorMap& mapAh,
+                        const GemmParams& p, int num_sms, cudaStream_t stream) {
   const int64_t max_pieces = p.R / Geo<PAIR>::PIECE + std::min(p.E, p.R);
   const int64_t max_tiles = max_pieces * p.n_tiles;
   const size_t smem = smem_bytes_for<PAIR>(p.E);
@@ -827,8 +832,8 @@ cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
   if (err != cudaSuccess) return err;
   if constexpr (PAIR == 1) {
     const int grid = static_cast<int>(std::min<int64_t>(max_tiles, num_sms));
-    grouped_gemm_kernel<MODE, 1, false><<<grid, NUM_THREADS, smem, stream>>>(mapA, mapB, mapA, mapB, p, p, nullptr,
-                                                                              nullptr);
+    grouped_gemm_kernel<MODE, 1, false><<<grid, NUM_THREADS, smem, stream>>>(mapA, mapB, mapA, mapB, mapAh, mapAh, p,
+                                                                              p, nullptr, nullptr);
     return cudaGetLastError();
   } else {
     const int clusters =
@@ -845,7 +850,8 @@ cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 2, false>, mapA, mapB, mapA, mapB, p, p,
+    // (a CTA pair has no half tiles: the half maps are not read)
+    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 2, false>, mapA, mapB, mapA, mapB, mapAh, mapAh, p, p,
                               static_cast<int*>(nullptr), static_cast<int*>(nullptr));
   }
 }
@@ -885,7 +891,8 @@ bool encode_one_box_b(const GroupedGemmArgs& a, CUtensorMap* map, bool pair) {
 }
 
 template <int MODE>
-cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& mapB, GemmParams& p, bool pair) {
+cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& mapAh, CUtensorMap& mapB, GemmParams& p,
+                    bool pair) {
   const bool down = MODE == MODE_DOWN;
   const int K = down ? a.D : a.H;
   {
@@ -895,6 +902,8 @@ cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& ma
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
     const cuuint32_t box[2] = {64, BM};
     if (!encode_bf16_map(&mapA, a.A, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    const cuuint32_t half_box[2] = {64, HALF_ROWS};
+    if (!encode_bf16_map(&mapAh, a.A, 2, dims, strides, half_box)) return cudaErrorInvalidValue;
   }
   const cuuint64_t H = a.H, D = a.D, E = a.E;
   p.b_one_box = one_box_enabled() && encode_one_box_b<MODE>(a, &mapB, pair) ? 1 : 0;
@@ -952,13 +961,13 @@ cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& ma
 template <int MODE>
 cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t stream) {
   if (a.R == 0) return cudaSuccess;
-  CUtensorMap mapA, mapB;
+  CUtensorMap mapA, mapAh, mapB;
   GemmParams p;
   const int pair = choose_pair(a.R, a.E);
-  cudaError_t err = prepare<MODE>(a, mapA, mapB, p, pair == 2);
+  cudaError_t err = prepare<MODE>(a, mapA, mapAh, mapB, p, pair == 2);
   if (err != cudaSuccess) return err;
-  if (pair == 2) return launch_with<MODE, 2>(mapA, mapB, p, a.num_sms, stream);
-  return launch_with<MODE, 1>(mapA, mapB, p, a.num_sms, stream);
+  if (pair == 2) return launch_with<MODE, 2>(mapA, mapB, mapAh, p, a.num_sms, stream);
+  return launch_with<MODE, 1>(mapA, mapB, mapAh, p, a.num_sms, stream);
 }
 
 // Rows per expert at which one bf16 weight byte carries as many FLOPs (2 per
@@ -970,11 +979,11 @@ template <int MODE>
 cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down, int* arrivals,
                          cudaStream_t stream) {
   if (up.R == 0) return cudaSuccess;
-  CUtensorMap mapA, mapB, mapA2, mapB2;
+  CUtensorMap mapA, mapAh, mapB, mapA2, mapA2h, mapB2;
   GemmParams p, p2;
-  cudaError_t err = prepare<MODE>(up, mapA, mapB, p, false);
+  cudaError_t err = prepare<MODE>(up, mapA, mapAh, mapB, p, false);
   if (err != cudaSuccess) return err;
-  err = prepare<MODE_DOWN>(down, mapA2, mapB2, p2, false);
+  err = prepare<MODE_DOWN>(down, mapA2, mapA2h, mapB2, p2, false);
   if (err != cudaSuccess) return err;
   // a timeout anywhere in the fused launch is reported as both stages'
   p.err_bit = p2.err_bit = MOE_DEVICE_ERR_TIMEOUT_GEMM1 | MOE_DEVICE_ERR_TIMEOUT_GEMM2;
@@ -1007,8 +1016,8 @@ cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down,
     if (env[0] == 's') dynamic = false;
   }
   int* sched = dynamic ? arrivals + mega_ffn_counters(up.R, up.E) - 1 : nullptr;
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 1, true>, mapA, mapB, mapA2, mapB2, p, p2, arrivals,
-                            sched);
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 1, true>, mapA, mapB, mapA2, mapB2, mapAh, mapA2h, p, p2,
+                            arrivals, sched);
 }
 
 }  // namespace
