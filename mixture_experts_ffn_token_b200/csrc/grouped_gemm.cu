@@ -586,9 +586,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             } else if constexpr (MODE == MODE_GATE_UP_CONCAT) {
               // leader: the 128 gate columns; peer: the matching 128 up columns
               const int c0 = tc.n * 128;
-              const int half = static_cast<int>(rank);
-              tma_load_4d_pair(sb, &mapB, fb, c0, half, kc, tc.e);
-              tma_load_4d_pair(sb + B_BOX_BYTES, &mapB, fb, c0 + 64, half, kc, tc.e);
+              const int gu = static_cast<int>(rank);  // 0: gate half, 1: up half
+              tma_load_4d_pair(sb, &mapB, fb, c0, gu, kc, tc.e);
+              tma_load_4d_pair(sb + B_BOX_BYTES, &mapB, fb, c0 + 64, gu, kc, tc.e);
             } else {
               const int c0 = tc.n * BN + static_cast<int>(rank) * 128;
               tma_load_3d_pair(sb, &mapB, fb, c0, kc, tc.e);
