@@ -39,8 +39,8 @@
 // piece starts once all gate_up tiles of that piece have published their h
 // (per-piece arrival counters, release/acquire).  CTAs take tiles with a
 // static stride or, below 256 rows per expert, from an atomic counter.  A
-// variant on CTA pairs (tcgen05 cta_group::2, 256x256 tiles, two launches)
-// is kept selectable.
+// variant on CTA pairs (tcgen05 cta_group::2, 256x256 tiles, M = 128 over
+// the pair for pieces of at most 128 rows, two launches) is kept selectable.
 //
 // Weights are read in their stored [K, N] (N-contiguous) layout: the B
 // operand is MN-major, which tcgen05 supports for 16-bit types, so no
@@ -93,6 +93,9 @@ struct Geo {
 constexpr int HALF_ROWS = 64;
 constexpr int HALF_A_BYTES = HALF_ROWS * BK * 2;  // 8 KB: the A rows a half tile copies
 constexpr uint32_t IDESC_HALF = idesc_bf16_f32(HALF_ROWS, BN, /*a_mn_major=*/false, /*b_mn_major=*/true);
+// CTA-pair tails: M = 128 over the pair (64 rows in each CTA); the
+// accumulator layout is given with kPairTail below.
+constexpr uint32_t IDESC_PAIR_TAIL = idesc_bf16_f32(BM, BN, /*a_mn_major=*/false, /*b_mn_major=*/true);
 
 constexpr int MODE_GATE_UP_CONCAT = 0;
 constexpr int MODE_GATE_UP_INTERLEAVED = 1;
@@ -226,19 +229,22 @@ constexpr int kStageRowBytes = 80;
 constexpr int kStageWarpBytes = 32 * kStageRowBytes;  // 2560 B per epilogue warp
 constexpr int kOutChunk = 32;                          // output columns per chunk
 
-// gate_up: 32 h columns starting at tile h column hc (relative to the tile).
+// gate_up: 32 h columns starting at tile h column hc (relative to the tile),
+// whose accumulator columns start at TMEM column tcol: concatenated, gate
+// of h column hc + i at tcol + i and up at tcol + up_off + i; interleaved,
+// the (gate, up) pair at tcol + 2i, tcol + 2i + 1.
 template <int MODE>
 __device__ __forceinline__ void gate_up_chunk(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int hc,
-                                              uint32_t (&packed)[16]) {
+                                              int tcol, int up_off, uint32_t (&packed)[16]) {
   const int hcol0 = tc.n * 128 + hc;  // absolute h column of value 0
   const __nv_bfloat16* bg = p.bias != nullptr ? p.bias + static_cast<int64_t>(tc.e) * 2 * p.D : nullptr;
   uint32_t a0[32], a1[32];
   if constexpr (MODE == MODE_GATE_UP_CONCAT) {
-    tmem_ld32(tacc + hc, a0);         // gate columns
-    tmem_ld32(tacc + 128 + hc, a1);   // matching up columns
+    tmem_ld32(tacc + tcol, a0);           // gate columns
+    tmem_ld32(tacc + tcol + up_off, a1);  // matching up columns
   } else {
-    tmem_ld32(tacc + 2 * hc, a0);     // (gate, up) pairs of h columns hc .. hc+15
-    tmem_ld32(tacc + 2 * hc + 32, a1);  // ... and hc+16 .. hc+31
+    tmem_ld32(tacc + tcol, a0);       // (gate, up) pairs of h columns hc .. hc+15
+    tmem_ld32(tacc + tcol + 32, a1);  // ... and hc+16 .. hc+31
   }
   tmem_ld_wait();
 #pragma unroll
@@ -273,13 +279,14 @@ __device__ __forceinline__ void gate_up_chunk(const GemmParams& p, const TileCoo
   }
 }
 
-// down: 32 output columns starting at tile column oc: (acc + b_d[e]) * w.
-__device__ __forceinline__ void down_chunk(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int oc,
+// down: 32 output columns starting at tile column oc, accumulator columns
+// from TMEM column tcol: (acc + b_d[e]) * w.
+__device__ __forceinline__ void down_chunk(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int oc, int tcol,
                                            float wgt, uint32_t (&packed)[16]) {
   const int col0 = tc.n * BN + oc;
   const __nv_bfloat16* bd = p.bias != nullptr ? p.bias + static_cast<int64_t>(tc.e) * p.H : nullptr;
   uint32_t a[32];
-  tmem_ld32(tacc + oc, a);
+  tmem_ld32(tacc + tcol, a);
   tmem_ld_wait();
 #pragma unroll
   for (int j = 0; j < 32; j += 2) {
@@ -294,14 +301,34 @@ __device__ __forceinline__ void down_chunk(const GemmParams& p, const TileCoord&
   }
 }
 
-// One tile's epilogue for one warp: rows quad*32.., output columns of `part`.
-template <int MODE>
+// Accumulator shapes of a tile in this CTA's TMEM.
+//   kFull      128 rows in lanes 0..127, the tile's 256 columns in TMEM
+//              columns 0..255 (in the order of the stage's B tile);
+//   kHalf      M = 64 (one CTA): row r in lane 32*(r/16) + r%16;
+//   kPairTail  M = 128 over a CTA pair, 64 rows in each CTA: lanes 0..63
+//              hold its rows for tile columns 0..127 and lanes 64..127 the
+//              same rows for columns 128..255, both in TMEM columns 0..127.
+constexpr int kFull = 0;
+constexpr int kHalf = 1;
+constexpr int kPairTail = 2;
+
+// One tile's epilogue for one warp (TMEM lane quadrant `quad`, column part
+// `part` of two).  A CTA pair's concatenated gate_up tile holds, per CTA B
+// half, the gate and then the up columns of 64 h columns, so a gate and its
+// up share a TMEM lane in every shape.
+template <int MODE, int PAIR>
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int quad,
-                                              int part, int lane, uint8_t* stage, bool half) {
+                                              int part, int lane, uint8_t* stage, int shape) {
   constexpr bool kDown = MODE == MODE_DOWN;
-  // tile row held by this thread's TMEM lane (half tiles: lanes 0..15 of the quadrant)
-  const int row = half ? quad * 16 + lane : quad * 32 + lane;
-  const bool has_row = !half || lane < 16;
+  // tile row held by this thread's TMEM lane
+  int row = quad * 32 + lane;
+  bool has_row = true;
+  if (shape == kHalf) {
+    row = quad * 16 + lane;
+    has_row = lane < 16;
+  } else if (shape == kPairTail) {
+    row = (quad & 1) * 32 + lane;
+  }
   // destination row of this thread's tile row, or -1 if it is not stored
   int64_t dst = -1;
   float wgt = 0.f;
@@ -327,23 +354,49 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoo
     const int hi = __shfl_sync(0xffffffffu, static_cast<int>(dst >> 32), src_lane);
     my_dst[i] = (static_cast<int64_t>(hi) << 32) | static_cast<uint32_t>(lo);
   }
+  // this warp's output columns: n_chunks chunks of 32 from tile column rel0,
+  // their accumulator columns from TMEM column tcol0, tstep apart
+  const bool tail = shape == kPairTail;
+  int rel0, tcol0, n_chunks, tstep, up_off = 128;
+  if constexpr (kDown) {
+    rel0 = tail ? (quad >> 1) * 128 + part * 64 : part * 128;
+    tcol0 = tail ? part * 64 : rel0;
+    n_chunks = tail ? 2 : 4;
+    tstep = 32;
+  } else if constexpr (MODE == MODE_GATE_UP_CONCAT) {
+    rel0 = tail ? (quad >> 1) * 64 + part * 32 : part * 64;
+    n_chunks = tail ? 1 : 2;
+    tstep = 32;
+    if constexpr (PAIR == 2) {
+      up_off = 64;
+      tcol0 = tail ? part * 32 : part * 128;
+    } else {
+      tcol0 = rel0;
+    }
+  } else {
+    rel0 = tail ? (quad >> 1) * 64 + part * 32 : part * 64;
+    tcol0 = tail ? part * 64 : 2 * rel0;
+    n_chunks = tail ? 1 : 2;
+    tstep = 64;
+  }
   const int limit = kDown ? p.H : p.D;
-  const int part_cols = kDown ? BN / 2 : 64;  // output columns per part
-  const int base_col = (kDown ? tc.n * BN : tc.n * 128) + part * part_cols;
+  const int base_col = kDown ? tc.n * BN : tc.n * 128;
   const int q = lane & 3;  // 16-byte chunk of a 64-byte row segment
   uint8_t* my_row = stage + lane * kStageRowBytes;
 #pragma unroll 1
-  for (int oc = 0; oc < part_cols; oc += kOutChunk) {
+  for (int ch = 0; ch < n_chunks; ++ch) {
+    const int rel = rel0 + kOutChunk * ch;
+    const int tcol = tcol0 + tstep * ch;
     uint32_t packed[16];
     __syncwarp();
-    if constexpr (kDown) down_chunk(p, tc, tacc, part * part_cols + oc, wgt, packed);
-    else gate_up_chunk<MODE>(p, tc, tacc, part * part_cols + oc, packed);
+    if constexpr (kDown) down_chunk(p, tc, tacc, rel, tcol, wgt, packed);
+    else gate_up_chunk<MODE>(p, tc, tacc, rel, tcol, up_off, packed);
 #pragma unroll
     for (int c = 0; c < 4; ++c)
       *reinterpret_cast<uint4*>(my_row + 16 * c) =
           make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
     __syncwarp();
-    const int col = base_col + oc + 8 * q;
+    const int col = base_col + rel + 8 * q;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int rr = 8 * i + (lane >> 2);
@@ -510,10 +563,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool ph2 = FUSED && t >= total1;
         const TileCoord tc = ph2 ? decode_tile(t - total1, p2.n_tiles, p.E, s_mt, s_off, G::PIECE)
                                  : decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
-        const int arow = (!ph2 && p.a_direct ? tc.row0 - s_off[tc.e] : tc.row0) + static_cast<int>(rank) * BM;
+        // a CTA pair's piece of at most 128 rows runs M = 128: 64 rows in each CTA
+        const bool pair_tail = PAIR == 2 && tc.rows <= BM;
+        const int arow = (!ph2 && p.a_direct ? tc.row0 - s_off[tc.e] : tc.row0) +
+                         static_cast<int>(rank) * (pair_tail ? HALF_ROWS : BM);
         const int nkb = ph2 ? p2.num_kb : p.num_kb;
         // a half tile (at most 64 rows, M = 64 MMAs) copies only 64 rows of A
-        const bool half = PAIR == 1 && tc.rows <= HALF_ROWS;
+        const bool half = (PAIR == 1 && tc.rows <= HALF_ROWS) || pair_tail;
         const uint32_t stage_tx = half ? G::STAGE_BYTES - HALF_A_BYTES : G::STAGE_BYTES;
         if constexpr (FUSED) {
           if (ph2) {
@@ -573,22 +629,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           } else {
             // The leader expects both CTAs' bytes on its own barrier; each
-            // CTA loads its 128 rows of A and its half of the 256 columns.
-            if (leader) mbar_arrive_expect_tx(full0 + 8 * s, 2 * G::STAGE_BYTES);
-            tma_load_2d_pair(sa, &mapA, fb, kc, arow);
+            // CTA loads its rows of A (128, or 64 in a tail) and its half of
+            // the 256 columns.
+            if (leader) mbar_arrive_expect_tx(full0 + 8 * s, 2 * stage_tx);
+            tma_load_2d_pair(sa, half ? &mapAh : &mapA, fb, kc, arow);
             if (p.b_one_box) {
               // this CTA's two 64-column blocks in one copy (concatenated:
-              // the leader's gate half, the peer's up half)
+              // the gate and the up block of h columns 64*rank .. +63 of the tile)
               if constexpr (MODE == MODE_GATE_UP_CONCAT)
-                tma_load_5d_pair(sb, &mapB, fb, 0, kc, 2 * tc.n, static_cast<int>(rank), tc.e);
+                tma_load_5d_pair(sb, &mapB, fb, 0, kc, 2 * tc.n + static_cast<int>(rank), 0, tc.e);
               else
                 tma_load_4d_pair(sb, &mapB, fb, 0, kc, 4 * tc.n + 2 * static_cast<int>(rank), tc.e);
             } else if constexpr (MODE == MODE_GATE_UP_CONCAT) {
-              // leader: the 128 gate columns; peer: the matching 128 up columns
-              const int c0 = tc.n * 128;
-              const int gu = static_cast<int>(rank);  // 0: gate half, 1: up half
-              tma_load_4d_pair(sb, &mapB, fb, c0, gu, kc, tc.e);
-              tma_load_4d_pair(sb + B_BOX_BYTES, &mapB, fb, c0 + 64, gu, kc, tc.e);
+              // the gate and the up block of h columns c0 .. c0+63
+              const int c0 = tc.n * 128 + 64 * static_cast<int>(rank);
+              tma_load_4d_pair(sb, &mapB, fb, c0, 0, kc, tc.e);
+              tma_load_4d_pair(sb + B_BOX_BYTES, &mapB, fb, c0, 1, kc, tc.e);
             } else {
               const int c0 = tc.n * BN + static_cast<int>(rank) * 128;
               tma_load_3d_pair(sb, &mapB, fb, c0, kc, tc.e);
@@ -642,10 +698,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool ph2 = FUSED && t >= total1;
         const int nkb = ph2 ? p2.num_kb : p.num_kb;
         uint32_t idesc = G::IDESC;
-        if constexpr (PAIR == 1) {
+        {
           const TileCoord tc = ph2 ? decode_tile(t - total1, p2.n_tiles, p.E, s_mt, s_off, G::PIECE)
                                    : decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
-          if (tc.rows <= HALF_ROWS) idesc = IDESC_HALF;
+          if (PAIR == 1 && tc.rows <= HALF_ROWS) idesc = IDESC_HALF;
+          if (PAIR == 2 && tc.rows <= BM) idesc = IDESC_PAIR_TAIL;
         }
         for (int kb = 0; kb < nkb; ++kb) {
           const int s = it % G::STAGES;
@@ -665,7 +722,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // B: N-major; 64-column blocks B_BOX_BYTES apart (LBO), 8-row K
             // groups 1024 B apart (SBO); a 16-row K step is 2048 B.
             const uint64_t b_desc = smem_desc_sw128(sb + kk * UMMA_K * 128, B_BOX_BYTES, 1024);
-            if constexpr (PAIR == 2) mma_bf16_ss_pair(d_tmem, a_desc, b_desc, G::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            if constexpr (PAIR == 2) mma_bf16_ss_pair(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
             else mma_bf16_ss(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           if constexpr (PAIR == 2) mma_commit_pair(empty0 + 8 * s, 0x3);
@@ -697,9 +754,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool ph2 = FUSED && t >= total1;
       TileCoord tc = ph2 ? decode_tile(t - total1, p2.n_tiles, p.E, s_mt, s_off, G::PIECE)
                          : decode_tile(t, p.n_tiles, p.E, s_mt, s_off, G::PIECE);
-      if constexpr (PAIR == 2) {
-        tc.row0 += static_cast<int>(rank) * BM;
-        tc.rows -= static_cast<int>(rank) * BM;  // may be <= 0: nothing of this half is stored
+      int shape = kFull;
+      if constexpr (PAIR == 1) {
+        if (tc.rows <= HALF_ROWS) shape = kHalf;
+      } else {
+        // a piece of at most 128 rows: M = 128 over the pair, 64 rows each
+        const int share = tc.rows <= BM ? HALF_ROWS : BM;
+        if (tc.rows <= BM) shape = kPairTail;
+        tc.row0 += static_cast<int>(rank) * share;
+        tc.rows -= static_cast<int>(rank) * share;  // may be <= 0: nothing of this half is stored
       }
       const int acc = ti & 1;
       const uint32_t aph = static_cast<uint32_t>(ti >> 1) & 1u;
@@ -708,11 +771,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after_sync();
       const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quad * 32) << 16);
       uint8_t* stage = s_stage + (warp - 2) * kStageWarpBytes;
-      const bool half = PAIR == 1 && tc.rows <= HALF_ROWS;
       if (ph2) {
-        epilogue_tile<MODE_DOWN>(p2, tc, tacc, quad, part, lane, stage, half);
+        epilogue_tile<MODE_DOWN, PAIR>(p2, tc, tacc, quad, part, lane, stage, shape);
       } else {
-        epilogue_tile<MODE>(p, tc, tacc, quad, part, lane, stage, half);
+        epilogue_tile<MODE, PAIR>(p, tc, tacc, quad, part, lane, stage, shape);
         if constexpr (FUSED) {
           // publish this warp's h stores of the piece to the down tiles
           fence_proxy_async_global();
@@ -850,7 +912,7 @@ cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // (a CTA pair has no half tiles: the half maps are not read)
+    // (the pair's tails of at most 128 rows copy 64 A rows per CTA through mapAh)
     return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 2, false>, mapA, mapB, mapA, mapB, mapAh, mapAh, p, p,
                               static_cast<int*>(nullptr), static_cast<int*>(nullptr));
   }
@@ -873,7 +935,9 @@ bool encode_one_box_b(const GroupedGemmArgs& a, CUtensorMap* map, bool pair) {
     if (D % 64 != 0) return false;
     const cuuint64_t dims[5] = {64, H, D / 64, 2, E};
     const cuuint64_t strides[4] = {2 * D * 2, 128, D * 2, H * 2 * D * 2};
-    const cuuint32_t box[5] = {64, BK, 2, pair ? 1u : 2u, 1};
+    // one CTA: both 64-column blocks of the gate half, then of the up half;
+    // a CTA of a pair: the gate and the up block of its 64 h columns
+    const cuuint32_t box[5] = {64, BK, pair ? 1u : 2u, 2, 1};
     return encode_bf16_map(map, a.W, 5, dims, strides, box);
   } else if (MODE == MODE_GATE_UP_INTERLEAVED) {
     if ((2 * D) % 64 != 0) return false;
