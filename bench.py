@@ -60,11 +60,13 @@ def max_over_ranks(x, dist_mod, device):
 def launches_per_step(wl, single_launch):
     """Kernels one call launches: router + 3-kernel CSR build (one kernel
     when T*k <= 2048 and E <= 512), gather, the two grouped GEMMs (one
-    launch when fused), combine, and with shared experts their index,
-    gather and GEMMs."""
+    launch when fused), combine, and with shared experts their index and
+    GEMMs (plus their gather only when the router weight scales the input:
+    otherwise their gate_up GEMM reads x directly)."""
     small = wl.num_tokens * wl.top_k <= 2048 and wl.num_experts <= 512
     gemms = 1 if single_launch else 2
-    return (1 if small else 4) + 1 + gemms + ((2 + gemms) if wl.num_shared > 0 else 0) + 1
+    shared = (1 + (1 if wl.weight_first else 0) + gemms) if wl.num_shared > 0 else 0
+    return (1 if small else 4) + 1 + gemms + shared + 1
 
 
 def job_throughput(world, tokens_per_rank, ms_per_step):
