@@ -361,6 +361,24 @@ def test_forward_full_size_sampled(name):
     run_and_check(wl, seed=0, device_inputs=True, sample_tokens=sample)
 
 
+@pytest.mark.parametrize("name,order", [("gptoss", "dynamic"), ("sink", "static"), ("sink", "dynamic")])
+def test_full_size_runs_are_bit_identical(name, order, monkeypatch):
+    """Which CTA computes which tile changes from run to run (the dynamic
+    order draws tiles from an atomic counter); what each tile computes, and
+    the combine's summation order, do not: repeated full-size calls give the
+    same bits, in the workload's default tile order and in the other."""
+    monkeypatch.setenv("MOE_B200_TILE_SCHEDULE", order)
+    wl = WORKLOADS[name]
+    d = to_dev(make_inputs(wl, 21, device="cuda"))
+    first = GpuRun(wl, d)
+    assert first.status == 0
+    for _ in range(2):
+        again = GpuRun(wl, d)
+        assert again.status == 0
+        assert torch.equal(first.out, again.out) and torch.equal(first.idx, again.idx)
+        assert torch.equal(first.w, again.w)
+
+
 def test_nvtx_ranges_change_nothing():
     """With MOE_B200_NVTX=1 (read once per process) every API call and kernel
     enqueue is wrapped in an NVTX range; the layer still matches the oracle."""
