@@ -38,6 +38,9 @@ UNIT = "tokens/s"
 DEFAULT_CONFIG = "mixtral"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# the B200 data-sheet figures, for context beside the measured fractions:
+# dense bf16 tensor throughput and HGX HBM3e bandwidth
+NOMINAL_PEAKS = {"TFLOP/s": 2250.0, "GB/s": 7700.0}
 
 
 # ------------------------------------------------------------------ helpers
@@ -298,7 +301,7 @@ def run_reference(args, wl):
         "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_block(wl, world),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "cpu_model": cpu_model(),
                          "sample": f"{n} of {wl.num_tokens} tokens per step (router + expert FFN, fp64)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -615,6 +618,7 @@ def run_gpu(args, wl):
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "peak_kind": f"{peak_kind} hbm copy"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["frac_of_nominal"] = roof["achieved"] / NOMINAL_PEAKS[roof["unit"]]
     roof["kernel"] = dom_name
     roof["traffic"] = kernel_traffic(wl.name, dom_name)
     roof["kernel_ms"] = kernel_ms                # live, in the timed region
@@ -647,10 +651,22 @@ def run_gpu(args, wl):
     return 0
 
 
+def cpu_model():
+    """The host CPU's model name (Linux), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_baseline(wl, inp):
     host = host_copy_for_oracle(inp)
     n, rate, dt, threads = calibrated_sample(wl, host, 15.0)
-    return {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+    return {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"{n} of {wl.num_tokens} tokens (router + expert FFN, fp64), {dt:.1f} s"}
 
 
