@@ -145,7 +145,7 @@ def test_forward_tiny_seeds(seed):
     run_and_check(WORKLOADS["tiny"], seed=seed)
 
 
-@pytest.mark.parametrize("variant", [
+EDGE_CASES = [
     dict(num_tokens=1), dict(top_k=1), dict(num_tokens=3, top_k=8), dict(num_experts=37, logits_std=1.0),
     dict(num_experts=64, num_tokens=4),                         # most experts empty
     dict(gate_up_format="interleaved"), dict(activation="gelu_tanh"),
@@ -157,8 +157,19 @@ def test_forward_tiny_seeds(seed):
     dict(num_experts=1024, top_k=32, num_tokens=40, logits_std=1.0),  # the library's largest E and k
     dict(num_tokens=64, hidden_dim=8192, moe_dim=64),           # long gate_up K (128 K blocks), tiny down K
     dict(num_tokens=48, hidden_dim=64, moe_dim=8192),           # long down K, 64 gate_up column blocks
-])
+]
+
+
+@pytest.mark.parametrize("variant", EDGE_CASES)
 def test_forward_edge_cases(variant):
+    run_and_check(WORKLOADS["tiny"].replace(**variant), seed=3)
+
+
+@pytest.mark.parametrize("variant", EDGE_CASES)
+def test_forward_edge_cases_cta_pair(variant, monkeypatch):
+    """The same shapes on CTA pairs: 256-row pieces, tails of at most 128
+    rows as M = 128 pair MMAs, gate/up-paired B halves."""
+    set_variant(monkeypatch, "two_launches_cta_pair")
     run_and_check(WORKLOADS["tiny"].replace(**variant), seed=3)
 
 
