@@ -29,20 +29,33 @@ def test_token_mask(wl):
     run_and_check_ex(wl.replace(mask_frac=0.3), seed=2)
 
 
+# GEMM variants (the default single launch, two launches, CTA pairs): the
+# shared experts' gate_up GEMM reads x directly in each of them.
+GEMM_VARIANTS = {"single_launch": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1"},
+                 "two_launches": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "1"},
+                 "cta_pair": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "2"}}
+
+
+@pytest.mark.parametrize("variant", sorted(GEMM_VARIANTS))
 @pytest.mark.parametrize("wl", [SNK.replace(num_shared=2, shared_dim=136),
                                 MIX.replace(num_shared=1, shared_dim=256),
                                 GPT.replace(num_shared=1, shared_dim=96),
                                 SNK.replace(num_tokens=1200, num_shared=2, shared_dim=72)],
                          ids=["sink_gated", "softmax_ungated", "gpt_bias", "sink_big"])
-def test_shared_experts(wl):
+def test_shared_experts(wl, variant, monkeypatch):
+    for k, v in GEMM_VARIANTS[variant].items():
+        monkeypatch.setenv(k, v)
     run_and_check_ex(wl, seed=3)
 
 
-@pytest.mark.parametrize("single_launch", ["1", "0"])
-def test_everything_together(single_launch, monkeypatch):
-    monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", single_launch)
+@pytest.mark.parametrize("variant", sorted(GEMM_VARIANTS))
+def test_everything_together(variant, monkeypatch):
+    for k, v in GEMM_VARIANTS[variant].items():
+        monkeypatch.setenv(k, v)
     run_and_check_ex(SNK.replace(num_shared=2, shared_dim=136, weight_first=True, mask_frac=0.25), seed=4)
     run_and_check_ex(GPT.replace(num_shared=1, shared_dim=200, weight_first=True, mask_frac=0.5), seed=5)
+    # shared experts reading x directly (no router weight first), with a mask
+    run_and_check_ex(SNK.replace(num_shared=2, shared_dim=136, mask_frac=0.25), seed=6)
 
 
 def test_no_extras_equals_forward():
