@@ -372,6 +372,18 @@ def test_forward_full_size_sampled(name):
     run_and_check(wl, seed=0, device_inputs=True, sample_tokens=sample)
 
 
+@pytest.mark.parametrize("name", ["mixtral", "sink"])
+def test_forward_full_size_sampled_cta_pair(name, monkeypatch):
+    """The selectable CTA-pair variant at full size: 256-row pieces and
+    M = 128 pair tails over every expert of the workload."""
+    set_variant(monkeypatch, "two_launches_cta_pair")
+    wl = WORKLOADS[name]
+    T = wl.num_tokens
+    rng = np.random.default_rng(124)
+    sample = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=min(T, FULL_SAMPLE), replace=False)]))
+    run_and_check(wl, seed=0, device_inputs=True, sample_tokens=sample)
+
+
 @pytest.mark.parametrize("name,order", [("gptoss", "dynamic"), ("sink", "static"), ("sink", "dynamic")])
 def test_full_size_runs_are_bit_identical(name, order, monkeypatch):
     """Which CTA computes which tile changes from run to run (the dynamic
