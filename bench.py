@@ -651,6 +651,25 @@ def run_gpu(args, wl):
     return 0
 
 
+def apply_overrides(wl, items):
+    """The workload with each FIELD=VALUE of `items` applied (converted to the
+    field's type) and its name extended by them, so that a changed workload
+    never picks up figures recorded for the named one."""
+    if not items:
+        return wl
+    kw = {}
+    for item in items:
+        field, sep, value = item.partition("=")
+        if not sep or field == "name" or not hasattr(wl, field):
+            raise SystemExit(f"--override: not a workload field assignment: {item!r}")
+        cur = getattr(wl, field)
+        if isinstance(cur, bool):
+            kw[field] = value.lower() in ("1", "true", "yes")
+        else:
+            kw[field] = type(cur)(value)
+    return wl.replace(name=wl.name + "+" + ",".join(items), **kw)
+
+
 def cpu_model():
     """The host CPU's model name (Linux), or None."""
     try:
@@ -682,10 +701,13 @@ def main():
                     help="streams per direction that share each e2e step's host<->device copies")
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="time replays of a CUDA graph of one step (default) or eager calls")
+    ap.add_argument("--override", action="append", default=[], metavar="FIELD=VALUE",
+                    help="change one field of the named workload (repeatable), e.g. moe_dim=7168; "
+                         "the line's workload name records every override")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    wl = WORKLOADS[args.config]
+    wl = apply_overrides(WORKLOADS[args.config], args.override)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_gpu(args, wl)

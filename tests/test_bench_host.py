@@ -53,3 +53,20 @@ def test_traffic_figures_are_used_only_for_the_captured_code():
             assert got == (ent["bytes_per_launch"] if current else None)
             assert ent["bytes_per_launch"] == ent["read"] + ent["write"]
     assert bench.kernel_traffic("no_such_workload", "mega_ffn") is None
+
+
+def test_workload_overrides():
+    from mixture_experts_ffn_token_b200.workloads import WORKLOADS
+    base = WORKLOADS["mixtral"]
+    wl = bench.apply_overrides(base, ["moe_dim=7168", "has_bias=true", "logits_std=0.5"])
+    assert (wl.moe_dim, wl.has_bias, wl.logits_std) == (7168, True, 0.5)
+    assert wl.name == "mixtral+moe_dim=7168,has_bias=true,logits_std=0.5"
+    # figures recorded for the named workload are not used for a changed one
+    assert bench.kernel_traffic(wl.name, "mega_ffn") is None
+    assert bench.apply_overrides(base, []) is base
+    for bad in (["moe_dim"], ["name=x"], ["no_such_field=1"]):
+        try:
+            bench.apply_overrides(base, bad)
+        except SystemExit:
+            continue
+        raise AssertionError(f"{bad} accepted")
