@@ -51,6 +51,13 @@ def dist_env():
     return world, rank, local
 
 
+def check_world(gpus, world):
+    """--gpus N must match the number of ranks the launcher started."""
+    if gpus != world:
+        raise SystemExit(f"--gpus {gpus} but {world} rank(s) were started: run N > 1 GPUs as "
+                         f"python -m torch.distributed.run --nproc-per-node {gpus} bench.py --gpus {gpus}")
+
+
 def max_over_ranks(x, dist_mod, device):
     """Max of a per-rank float over all ranks (identity without a process group)."""
     if dist_mod is None:
@@ -708,6 +715,7 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     wl = apply_overrides(WORKLOADS[args.config], args.override)
+    check_world(args.gpus, dist_env()[0])
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_gpu(args, wl)

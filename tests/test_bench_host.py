@@ -70,3 +70,15 @@ def test_workload_overrides():
         except SystemExit:
             continue
         raise AssertionError(f"{bad} accepted")
+
+
+def test_gpus_must_match_the_started_ranks():
+    bench.check_world(1, 1)
+    bench.check_world(4, 4)
+    for gpus, world in ((2, 1), (1, 2)):
+        try:
+            bench.check_world(gpus, world)
+        except SystemExit as e:
+            assert "torch.distributed.run" in str(e)
+            continue
+        raise AssertionError(f"--gpus {gpus} accepted with {world} rank(s)")
