@@ -51,6 +51,48 @@ def dist_env():
     return world, rank, local
 
 
+def roofline(wl, stage, kernel_ms, peaks, peak_kind, clock_summary, used_experts):
+    """The dominant stage's roofline entry: its algorithmic FLOPs (GEMM
+    stages) or bytes over its live time `kernel_ms`, against the peak that
+    bounds it. A GEMM stage is tensor-bound when its FLOPs at the bf16 peak
+    take longer than its touched experts' weight bytes at the HBM copy
+    bandwidth, else HBM-bound. The bf16 peak is the sustained figure when
+    NVML saw `sw_power_cap` during the timed region, the burst figure
+    otherwise."""
+    capped = "sw_power_cap" in clock_summary.get("reasons", [])
+    bf16_peak = peaks.get("bf16_tflops_sustained" if capped else "bf16_tflops", peaks.get("bf16_tflops"))
+    bf16_kind = "sustained" if capped else "burst"
+    T, k, H = wl.num_tokens, wl.top_k, wl.hidden_dim
+    gemm_stages = ("gemm_gate_up", "gemm_down", "shared_gemm_gate_up", "shared_gemm_down", "mega_ffn",
+                   "shared_mega_ffn")
+    if stage in gemm_stages:
+        # FLOP / weight-byte multipliers: gate_up 4 / 2, down 2 / 1, both 6 / 3
+        fm, bm = (6, 3) if stage.endswith("mega_ffn") else (4, 2) if stage.endswith("gate_up") else (2, 1)
+        if stage.startswith("shared"):
+            kflops = fm * T * wl.num_shared * H * wl.shared_dim
+            kbytes = bm * wl.num_shared * H * wl.shared_dim * 2
+        else:
+            kflops = fm * T * k * H * wl.moe_dim
+            kbytes = bm * used_experts * H * wl.moe_dim * 2
+        t_flop = kflops / (bf16_peak * 1e12)
+        t_byte = kbytes / (peaks["hbm_gbs"] * 1e9)
+        if t_flop >= t_byte:
+            achieved = kflops / (kernel_ms / 1e3) / 1e12
+            roof = {"bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
+                    "peak_kind": f"{peak_kind} bf16 {bf16_kind}"}
+        else:
+            achieved = kbytes / (kernel_ms / 1e3) / 1e9
+            roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "peak_kind": f"{peak_kind} hbm copy"}
+    else:
+        achieved = workload_bytes(wl) / (kernel_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "peak_kind": f"{peak_kind} hbm copy"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["frac_of_nominal"] = roof["achieved"] / NOMINAL_PEAKS[roof["unit"]]
+    return roof
+
+
 def check_world(gpus, world):
     """--gpus N must match the number of ranks the launcher started."""
     if gpus != world:
@@ -590,42 +632,9 @@ def run_gpu(args, wl):
                   "shared_gemm_down": "(shared fused)"}.get(n, n) for n in names]
     flops = wl.flops()
     wbytes, used = touched_expert_bytes(wl, idx)
-    shared_rows = T * wl.num_shared
     dom_name = names[dom]
     clock_summary = clocks.summary()
-    # a GEMM timed while the power cap held the clocks down is compared with
-    # the sustained bf16 figure, otherwise with the burst figure
-    capped = "sw_power_cap" in clock_summary.get("reasons", [])
-    bf16_peak = peaks.get("bf16_tflops_sustained" if capped else "bf16_tflops", peaks.get("bf16_tflops"))
-    bf16_kind = "sustained" if capped else "burst"
-    gemm_stages = ("gemm_gate_up", "gemm_down", "shared_gemm_gate_up", "shared_gemm_down", "mega_ffn",
-                   "shared_mega_ffn")
-    if dom_name in gemm_stages:
-        # FLOP / weight-byte multipliers: gate_up 4 / 2, down 2 / 1, both 6 / 3
-        fm, bm = (6, 3) if dom_name.endswith("mega_ffn") else (4, 2) if dom_name.endswith("gate_up") else (2, 1)
-        if dom_name.startswith("shared"):
-            kflops = fm * shared_rows * H * wl.shared_dim
-            kbytes = bm * wl.num_shared * H * wl.shared_dim * 2
-        else:
-            kflops = fm * T * k * H * wl.moe_dim
-            kbytes = bm * used * H * wl.moe_dim * 2
-        t_flop = kflops / (bf16_peak * 1e12)
-        t_byte = kbytes / (peaks["hbm_gbs"] * 1e9)
-        if t_flop >= t_byte:
-            achieved = kflops / (kernel_ms / 1e3) / 1e12
-            roof = {"bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
-                    "peak_kind": f"{peak_kind} bf16 {bf16_kind}"}
-        else:
-            achieved = kbytes / (kernel_ms / 1e3) / 1e9
-            roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "peak_kind": f"{peak_kind} hbm copy"}
-    else:
-        kb = workload_bytes(wl)
-        achieved = kb / (kernel_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "peak_kind": f"{peak_kind} hbm copy"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["frac_of_nominal"] = roof["achieved"] / NOMINAL_PEAKS[roof["unit"]]
+    roof = roofline(wl, dom_name, kernel_ms, peaks, peak_kind, clock_summary, used)
     roof["kernel"] = dom_name
     roof["traffic"] = kernel_traffic(wl.name, dom_name)
     roof["kernel_ms"] = kernel_ms                # live, in the timed region

@@ -82,3 +82,29 @@ def test_gpus_must_match_the_started_ranks():
             assert "torch.distributed.run" in str(e)
             continue
         raise AssertionError(f"--gpus {gpus} accepted with {world} rank(s)")
+
+
+def test_roofline_arithmetic():
+    """The dominant kernel's roofline entry: algorithmic FLOPs (or weight
+    bytes) over its time, against the peak that bounds it."""
+    from mixture_experts_ffn_token_b200.workloads import WORKLOADS
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    mix = WORKLOADS["mixtral"]
+    flops = 6 * 8192 * 4096 * 14336
+    r = bench.roofline(mix, "mega_ffn", 2.0, peaks, "measured", {"reasons": []}, 8)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["peak"] == 1600.0
+    assert abs(r["achieved"] - flops / 2e-3 / 1e12) < 1e-9 * r["achieved"]
+    assert abs(r["frac"] - r["achieved"] / 1600.0) < 1e-12
+    assert abs(r["frac_of_nominal"] - r["achieved"] / 2250.0) < 1e-12
+    # the power cap selects the sustained figure
+    capped = bench.roofline(mix, "mega_ffn", 2.0, peaks, "measured", {"reasons": ["sw_power_cap"]}, 8)
+    assert capped["peak"] == 1400.0 and "sustained" in capped["peak_kind"]
+    # 64 rows per expert (gptoss): the touched experts' weight bytes bound it
+    go = WORKLOADS["gptoss"]
+    g = bench.roofline(go, "mega_ffn", 1.0, peaks, "measured", {"reasons": []}, 128)
+    wbytes = 3 * 128 * 2880 * 2880 * 2
+    assert g["bound"] == "hbm" and g["unit"] == "GB/s"
+    assert abs(g["achieved"] - wbytes / 1e-3 / 1e9) < 1e-9 * g["achieved"]
+    # the gate_up GEMM alone (two launches): 4 R H D FLOPs
+    up = bench.roofline(mix, "gemm_gate_up", 1.0, peaks, "measured", {"reasons": []}, 8)
+    assert abs(up["achieved"] - 4 * 8192 * 4096 * 14336 / 1e-3 / 1e12) < 1e-9 * up["achieved"]
