@@ -51,17 +51,21 @@ def dist_env():
     return world, rank, local
 
 
-def roofline(wl, stage, kernel_ms, peaks, peak_kind, clock_summary, used_experts):
+def roofline(wl, stage, kernel_ms, peaks, peak_kind, clock_summary, used_experts, region_s=0.0):
     """The dominant stage's roofline entry: its algorithmic FLOPs (GEMM
     stages) or bytes over its live time `kernel_ms`, against the peak that
     bounds it. A GEMM stage is tensor-bound when its FLOPs at the bf16 peak
     take longer than its touched experts' weight bytes at the HBM copy
-    bandwidth, else HBM-bound. The bf16 peak is the sustained figure when
-    NVML saw `sw_power_cap` during the timed region, the burst figure
-    otherwise."""
+    bandwidth, else HBM-bound. `frac` is taken against the burst bf16 figure
+    (a timed region shorter than a second never settles at the power-capped
+    clock); only a region of a second or more that NVML saw under
+    `sw_power_cap` is compared with the sustained figure. `frac_sustained`
+    (the achieved rate over the sustained figure) is given beside it for
+    tensor-bound kernels."""
     capped = "sw_power_cap" in clock_summary.get("reasons", [])
-    bf16_peak = peaks.get("bf16_tflops_sustained" if capped else "bf16_tflops", peaks.get("bf16_tflops"))
-    bf16_kind = "sustained" if capped else "burst"
+    use_sustained = capped and region_s >= 1.0 and "bf16_tflops_sustained" in peaks
+    bf16_peak = peaks["bf16_tflops_sustained"] if use_sustained else peaks["bf16_tflops"]
+    bf16_kind = "sustained" if use_sustained else "burst"
     T, k, H = wl.num_tokens, wl.top_k, wl.hidden_dim
     gemm_stages = ("gemm_gate_up", "gemm_down", "shared_gemm_gate_up", "shared_gemm_down", "mega_ffn",
                    "shared_mega_ffn")
@@ -80,6 +84,8 @@ def roofline(wl, stage, kernel_ms, peaks, peak_kind, clock_summary, used_experts
             achieved = kflops / (kernel_ms / 1e3) / 1e12
             roof = {"bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
                     "peak_kind": f"{peak_kind} bf16 {bf16_kind}"}
+            if "bf16_tflops_sustained" in peaks:
+                roof["frac_sustained"] = achieved / peaks["bf16_tflops_sustained"]
         else:
             achieved = kbytes / (kernel_ms / 1e3) / 1e9
             roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -393,7 +399,7 @@ def timed_steps(step, steps, stream, flush):
     return total
 
 
-def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None, copy_streams=1):
+def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None, copy_streams=1, steps=None):
     """K steps of moe_forward (moe_forward_ex when `make_ex` builds its extras
     from a device token mask) fed from, and returning to, pinned host memory.
     The token mask, when there is one, is a per-step input and is copied too.
@@ -461,27 +467,39 @@ def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None, copy_streams=1):
         torch.cuda.synchronize()
         return start.elapsed_time(stop)
 
+    steps = args.steps if steps is None else steps
     region(max(2, args.warmup))
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    ms = region(args.steps)
-    if not torch.equal(out_h[(args.steps - 1) % 2], out_d[(args.steps - 1) % 2].cpu()):
+    ms = region(steps)
+    if not torch.equal(out_h[(steps - 1) % 2], out_d[(steps - 1) % 2].cpu()):
         raise RuntimeError("e2e: host copy of the output differs from the device result")
     return max_over_ranks(ms, dist, "cuda")
 
 
-def run_gpu(args, wl):
-    world, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
+def host_enqueue_us(step, calls, stream):
+    """Host microseconds per eager call of step(): the time the calling
+    thread spends in `calls` back-to-back calls (the Python binding, the
+    library's argument checks, tensor-map encoding and kernel launches).
+    Nothing in a call waits for the GPU; the device work is synchronized
+    afterwards, outside the timed interval."""
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        step()
+    t1 = time.perf_counter()
+    torch.cuda.synchronize()
+    return (t1 - t0) * 1e6 / calls
 
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    abi.load_library()
-    peaks, peak_kind = load_peaks()
+
+def measure(args, wl, ctx, steps):
+    """Every figure of one workload's bench line (without cpu_baseline):
+    warm-up, the stage region, the graph-timed region with the dominant
+    kernel's live events, the e2e region and the host enqueue cost.
+    Returns (line, inputs)."""
+    world, rank, local, dist = ctx["world"], ctx["rank"], ctx["local"], ctx["dist"]
+    peaks, peak_kind = ctx["peaks"], ctx["peak_kind"]
     cfg = abi.make_config(wl)
     inp = make_inputs(wl, seed=rank, device="cuda")
     T, H, k, S, E = wl.num_tokens, wl.hidden_dim, wl.top_k, wl.num_sink, wl.num_experts
@@ -521,7 +539,7 @@ def run_gpu(args, wl):
             flush.fill_(1)
     torch.cuda.synchronize()
     if abi.moe_device_status(ws) != 0:
-        raise RuntimeError("device status set during warm-up")
+        raise RuntimeError(f"{wl.name}: device status set during warm-up")
 
     # ---------------- stage region: K eager steps through moe_forward_timed,
     # each recording its own events between all stages (a timing event
@@ -529,17 +547,17 @@ def run_gpu(args, wl):
     # a breakdown, not the step time); it picks the dominant stage
     names = list(abi.STAGE_NAMES_EX if extras is not None else abi.STAGE_NAMES)
     n_ev = len(names) + 1
-    ev_sets = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    ev_sets = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(steps)]
     for evs in ev_sets:          # create the CUDA events outside the region
         for ev in evs:
             ev.record(stream)
     torch.cuda.synchronize()
     it = iter(ev_sets)
-    timed_steps(lambda: step(next(it)), args.steps, stream, flush)
-    stage_ms = [sum(evs[i].elapsed_time(evs[i + 1]) for evs in ev_sets) / args.steps for i in range(n_ev - 1)]
+    timed_steps(lambda: step(next(it)), steps, stream, flush)
+    stage_ms = [sum(evs[i].elapsed_time(evs[i + 1]) for evs in ev_sets) / steps for i in range(n_ev - 1)]
     dom = max(range(len(names)), key=lambda i: stage_ms[i])
     if abi.moe_device_status(ws) != 0:
-        raise RuntimeError("device status set during the stage region")
+        raise RuntimeError(f"{wl.name}: device status set during the stage region")
 
     # ---------------- timed region: K steps between two CUDA events on the
     # launching stream (max over ranks); L2 flushed between steps when the
@@ -553,9 +571,9 @@ def run_gpu(args, wl):
     def ext_event():  # recorded as an event node when captured in a graph
         return torch.cuda.Event(enable_timing=True, external=True)
 
-    pair_steps = [i for i in range(args.steps) if i % 10 == 9] or [args.steps - 1]
+    pair_steps = [i for i in range(steps) if i % 10 == 9] or [steps - 1]
     pairs = {i: (ext_event(), ext_event()) for i in pair_steps}
-    marks = [(ext_event(), ext_event()) for _ in range(args.steps)]
+    marks = [(ext_event(), ext_event()) for _ in range(steps)]
     for a, b in list(pairs.values()) + marks:
         a.record(stream)
         b.record(stream)
@@ -569,7 +587,7 @@ def run_gpu(args, wl):
         return evs
 
     def body():
-        for i in range(args.steps):
+        for i in range(steps):
             if flush is not None:
                 flush.fill_(1)
                 marks[i][0].record()
@@ -586,7 +604,7 @@ def run_gpu(args, wl):
         graph.replay()           # untimed warm replay
         torch.cuda.synchronize()
         if abi.moe_device_status(ws) != 0:
-            raise RuntimeError("device status set by the captured steps")
+            raise RuntimeError(f"{wl.name}: device status set by the captured steps")
         run = graph.replay
     if dist is not None:
         dist.barrier()
@@ -597,8 +615,9 @@ def run_gpu(args, wl):
         run()
         stop.record(stream)
         torch.cuda.synchronize()
+    region_ms = start.elapsed_time(stop)
     if flush is None:
-        elapsed_ms = start.elapsed_time(stop)
+        elapsed_ms = region_ms
     else:
         elapsed_ms = sum(a.elapsed_time(b) for a, b in marks)
     kernel_ms = sum(a.elapsed_time(b) for a, b in pairs.values()) / len(pairs)
@@ -607,21 +626,26 @@ def run_gpu(args, wl):
     torch.cuda.synchronize()
     status = abi.moe_device_status(ws)
     if status != 0:
-        raise RuntimeError(f"device status {status:#x} after the timed region")
+        raise RuntimeError(f"{wl.name}: device status {status:#x} after the timed region")
     elapsed_ms = max_over_ranks(elapsed_ms, dist, "cuda")
-    ms_per_step = elapsed_ms / args.steps
+    ms_per_step = elapsed_ms / steps
     value = job_throughput(world, T, ms_per_step)
+    del graph
 
     # ---------------- e2e: host buffers; every step copies its inputs host->device
     # from pinned memory and its output device->host inside the timed region.
     # Copies run on their own streams, double-buffered, so step i's copies
     # overlap the compute of its neighbours.
-    e2e_ms = run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex, copy_streams=args.copy_streams)
-    e2e_value = job_throughput(world, T, e2e_ms / args.steps)
+    e2e_ms = run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex, copy_streams=args.copy_streams, steps=steps)
+    e2e_value = job_throughput(world, T, e2e_ms / steps)
     x_h_bytes = inp["x"].numel() * 2 + inp["logits"].numel() * 4
     if inp["token_mask"] is not None:
         x_h_bytes += inp["token_mask"].numel()
     out_bytes = T * H * 2
+
+    # ---------------- host cost of one eager call (the public Python entry
+    # point and the library's enqueue work, no GPU wait)
+    host_us = host_enqueue_us(step, min(steps, 20), stream)
 
     # ---------------- roofline of the dominant kernel, timed live by its event
     # pair in the timed region
@@ -634,14 +658,14 @@ def run_gpu(args, wl):
     wbytes, used = touched_expert_bytes(wl, idx)
     dom_name = names[dom]
     clock_summary = clocks.summary()
-    roof = roofline(wl, dom_name, kernel_ms, peaks, peak_kind, clock_summary, used)
+    roof = roofline(wl, dom_name, kernel_ms, peaks, peak_kind, clock_summary, used, region_s=region_ms / 1e3)
     roof["kernel"] = dom_name
     roof["traffic"] = kernel_traffic(wl.name, dom_name)
     roof["kernel_ms"] = kernel_ms                # live, in the timed region
     roof["kernel_ms_stage_region"] = stage_ms[dom]
 
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random-init expert weights N(0,0.02))",
         "config": config_block(wl, world, graph=args.graph),
@@ -652,13 +676,55 @@ def run_gpu(args, wl):
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x_h_bytes,
                 "d2h_bytes_per_step": out_bytes},
-        "gpu_launches": launches_per_step(wl, fused) * args.steps,
+        "host_us_per_call": host_us,
+        "gpu_launches": launches_per_step(wl, fused) * steps,
         "single_launch_ffn": fused,
         "clocks": clock_summary,
     }
-    del graph
+    return line, inp
+
+
+# the other workloads of the per-config object, measured after the headline one
+PER_CONFIG = ("tiny", "gptoss", "sink", "decode")
+
+
+def compact(line):
+    """The per-config entry: the figures of a full line that describe one workload."""
+    keep = ("value", "unit", "ms_per_step", "steps", "tflops", "weight_gbs", "experts_touched", "roofline", "e2e",
+            "host_us_per_call", "gpu_launches", "clocks", "stages_ms")
+    ent = {k: line[k] for k in keep}
+    ent["workload"] = line["config"]["workload"]
+    ent["l2"] = line["config"]["l2"]
+    return ent
+
+
+def run_gpu(args, wl):
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    abi.load_library()
+    peaks, peak_kind = load_peaks()
+    ctx = {"world": world, "rank": rank, "local": local, "dist": dist, "peaks": peaks, "peak_kind": peak_kind}
+    line, inp = measure(args, wl, ctx, args.steps)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, inp)
+    del inp
+    per_config = args.per_config if args.per_config is not None else world == 1
+    if per_config:
+        line["per_config"] = {}
+        for name in PER_CONFIG:
+            if name == wl.name:
+                continue
+            torch.cuda.empty_cache()
+            sub, sub_inp = measure(args, WORKLOADS[name], ctx, args.steps)
+            del sub_inp
+            line["per_config"][name] = compact(sub)
+        torch.cuda.empty_cache()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -717,6 +783,9 @@ def main():
                     help="streams per direction that share each e2e step's host<->device copies")
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="time replays of a CUDA graph of one step (default) or eager calls")
+    ap.add_argument("--per-config", action=argparse.BooleanOptionalAction, default=None,
+                    help="also measure tiny, gptoss, sink and decode into the line's per_config object "
+                         "(default: on with one GPU, off with several)")
     ap.add_argument("--override", action="append", default=[], metavar="FIELD=VALUE",
                     help="change one field of the named workload (repeatable), e.g. moe_dim=7168; "
                          "the line's workload name records every override")

@@ -298,8 +298,16 @@ moe_status_t moe_forward_ex(const moe_config_t* cfg, const moe_extras_t* extras,
  * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  *
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  Every call shares the one array, which keeps
+ * (cudaGetSymbolAddress, with that device current) and caches it for the
+ * life of the process.  Under lazy module loading (CUDA_MODULE_LOADING=LAZY,
+ * the default) that lookup also loads the library module that holds the
+ * array, which places the 524,544 bytes in device memory and may
+ * synchronize the device: make the first call on each device once at
+ * initialisation, outside any stream capture and off the latency-critical
+ * path; later calls allocate and synchronize nothing.  The cached address
+ * belongs to the device's current primary context: after cudaDeviceReset
+ * (or anything else that destroys that context) it is stale, so no call may
+ * follow a context reset in the same process.  Every call shares the one array, which keeps
  * the last call's contents (the status word is cleared at the start of each
  * call, the tables are rewritten): calls that overlap on the GPU -- on two
  * streams, or from two threads -- race and give undefined results.  Device

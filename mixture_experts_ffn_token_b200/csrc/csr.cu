@@ -15,8 +15,9 @@
 //           the position of each slot, so the order inside an expert is the
 //           slot order and no atomic decides any position.
 #include <algorithm>
-
 #include <cstdlib>
+#include <mutex>
+#include <vector>
 
 #include "kernels.cuh"
 
@@ -181,6 +182,25 @@ bool pdl_enabled() {
   return !(env != nullptr && env[0] == '0');
 }
 
+cudaError_t opt_in_dynamic_smem(const void* func, int bytes) {
+  struct Done {
+    int dev;
+    const void* func;
+    cudaError_t result;
+  };
+  static std::mutex mu;
+  static std::vector<Done> done;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Done& d : done)
+    if (d.dev == dev && d.func == func) return d.result;
+  err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  done.push_back({dev, func, err});
+  return err;
+}
+
 namespace {
 
 constexpr int kCombineBatch = 8;   // rows a combine thread loads before summing
@@ -339,8 +359,9 @@ cudaError_t launch_csr_scatter(const int32_t* idx, int R, int E, const int32_t* 
   if (nchunks == 0) return cudaSuccess;
   const size_t smem = static_cast<size_t>(kCsrWarps) * E * sizeof(int);
   if (smem > 48 * 1024) {
-    cudaError_t err = cudaFuncSetAttribute(csr_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
+    // once per device, for the largest expert count
+    cudaError_t err = opt_in_dynamic_smem(reinterpret_cast<const void*>(csr_scatter_kernel),
+                                          static_cast<int>(static_cast<size_t>(kCsrWarps) * kMaxExperts * sizeof(int)));
     if (err != cudaSuccess) return err;
   }
   return launch_pdl(csr_scatter_kernel, dim3(nchunks), dim3(kCsrThreads), smem, stream, idx, R, E, chunk_base, perm,

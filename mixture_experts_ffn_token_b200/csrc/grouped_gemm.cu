@@ -836,14 +836,16 @@ constexpr size_t smem_bytes_for(int E) {
          2 * static_cast<size_t>(E + 1) * 4 + 16 + NUM_EPI_WARPS * kStageWarpBytes;
 }
 
-// Clusters of two that can be resident at once (cached per kernel).
+// Clusters of two that can be resident at once, looked up once per device
+// (occupancy depends on the device) and kernel.
 template <int MODE>
 int max_pair_clusters(size_t smem, int num_sms) {
-  // occupancy depends on the device: cached per device
   constexpr int kDevices = 64;
+  static std::mutex mu;
   static int cached[kDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) return num_sms / 2;
+  std::lock_guard<std::mutex> lock(mu);
   if (cached[dev] > 0) return cached[dev];
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -888,9 +890,8 @@ cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
   const int64_t max_pieces = p.R / Geo<PAIR>::PIECE + std::min(p.E, p.R);
   const int64_t max_tiles = max_pieces * p.n_tiles;
   const size_t smem = smem_bytes_for<PAIR>(p.E);
-  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, PAIR, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem_bytes_for<PAIR>(kMaxExperts)));
+  cudaError_t err = opt_in_dynamic_smem(reinterpret_cast<const void*>(grouped_gemm_kernel<MODE, PAIR, false>),
+                                        static_cast<int>(smem_bytes_for<PAIR>(kMaxExperts)));
   if (err != cudaSuccess) return err;
   if constexpr (PAIR == 1) {
     const int grid = static_cast<int>(std::min<int64_t>(max_tiles, num_sms));
@@ -1054,8 +1055,8 @@ cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down,
   const int64_t max_pieces = p.R / BM + std::min(p.E, p.R);
   const int64_t max_tiles = max_pieces * (p.n_tiles + p2.n_tiles);
   const size_t smem = smem_bytes_for<1>(p.E);
-  err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, 1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem_bytes_for<1>(kMaxExperts)));
+  err = opt_in_dynamic_smem(reinterpret_cast<const void*>(grouped_gemm_kernel<MODE, 1, true>),
+                            static_cast<int>(smem_bytes_for<1>(kMaxExperts)));
   if (err != cudaSuccess) return err;
   // Cooperative: the launch fails rather than run with CTAs that are not
   // resident, on which a down tile's wait could otherwise depend.

@@ -13,6 +13,13 @@ namespace moe {
 // touching global memory, so the overlap never changes what it reads.
 bool pdl_enabled();
 
+// Raises the dynamic shared-memory limit of kernel `func` to `bytes` on the
+// current device the first time it is asked for that (device, kernel); later
+// calls return the first call's result without calling the runtime.  Every
+// caller passes the kernel's largest possible size, so one opt-in serves all
+// launches.  Thread-safe.
+cudaError_t opt_in_dynamic_smem(const void* func, int bytes);
+
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                               Args... args) {

@@ -248,28 +248,15 @@ cudaError_t launch_small_npl(const RouterArgs& a, int32_t* offsets, int32_t* per
   const size_t smem = (kSmallSlots + static_cast<size_t>(kSmallWarps) * a.E) * sizeof(int);
   const dim3 block(32 * kSmallWarps);
   const dim3 one(1);
-  // the per-warp histograms need up to (2048 + 32 * 512) * 4 bytes, above the default 48 KB
-  // function attributes are per device: opt in once for each device
-  constexpr int kDevices = 64;
-  static bool opted_in[kDevices] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) return cudaErrorInvalidDevice;
-  if (!opted_in[dev]) {
-    const int max_smem = static_cast<int>((kSmallSlots + static_cast<size_t>(kSmallWarps) * kSmallExperts) * sizeof(int));
-    cudaError_t e =
-        cudaFuncSetAttribute(route_csr_small_kernel<NPL, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(route_csr_small_kernel<NPL, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               max_smem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(route_csr_small_kernel<NPL, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               max_smem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(route_csr_small_kernel<NPL, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               max_smem);
-    if (e != cudaSuccess) return e;
-    opted_in[dev] = true;
-  }
+  // the per-warp histograms need up to (2048 + 32 * 512) * 4 bytes, above
+  // the default 48 KB: opted in once per device and kernel
+  const int max_smem = static_cast<int>((kSmallSlots + static_cast<size_t>(kSmallWarps) * kSmallExperts) * sizeof(int));
+  const void* kernel = a.sink ? (a.logits_bf16 ? reinterpret_cast<const void*>(route_csr_small_kernel<NPL, true, true>)
+                                               : reinterpret_cast<const void*>(route_csr_small_kernel<NPL, true, false>))
+                              : (a.logits_bf16 ? reinterpret_cast<const void*>(route_csr_small_kernel<NPL, false, true>)
+                                               : reinterpret_cast<const void*>(route_csr_small_kernel<NPL, false, false>));
+  const cudaError_t e = opt_in_dynamic_smem(kernel, max_smem);
+  if (e != cudaSuccess) return e;
   if (a.sink) {
     if (a.logits_bf16)
       return launch_pdl(route_csr_small_kernel<NPL, true, true>, one, block, smem, stream, a, offsets, perm, status, mask);

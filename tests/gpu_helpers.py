@@ -13,6 +13,36 @@ WEIGHT_RTOL = 1e-5  # router weights (fp32) relative to the fp64 oracle
 WEIGHT_ATOL = 1e-30
 
 
+def every_tile_tokens(idx, num_experts, piece=128, token_mask=None):
+    """Token ids whose routed rows reach every tile of the grouped GEMMs.
+
+    A tile is (expert, row piece of `piece` permuted rows, output column
+    block), and a token's output row reads every column block of the pieces
+    its slots sit in, so one compared row per piece compares every tile of
+    both contractions.  Taken per expert segment of the CSR (slots sorted by
+    expert, stable; masked tokens' slots take no place): the first and last
+    row of every piece, and every row of the segment's last, ragged piece.
+    Pieces of 128 rows also cover the 256-row pieces of the CTA-pair
+    variant (each holds two of them)."""
+    idx = np.asarray(idx)
+    k = idx.shape[1]
+    flat = idx.reshape(-1)
+    slots = np.arange(flat.size)
+    if token_mask is not None:
+        slots = slots[np.asarray(token_mask)[slots // k] != 0]
+    order = slots[np.argsort(flat[slots], kind="stable")]
+    off = np.concatenate([[0], np.cumsum(np.bincount(flat[slots], minlength=num_experts))])
+    rows = []
+    for e in range(num_experts):
+        lo, hi = int(off[e]), int(off[e + 1])
+        for p0 in range(lo, hi, piece):
+            p1 = min(p0 + piece, hi)
+            rows += [p0, p1 - 1]
+            if p1 == hi:
+                rows += list(range(p0, p1))
+    return np.unique(order[np.asarray(rows, dtype=np.int64)] // k)
+
+
 def to_dev(inp, device="cuda"):
     return {k: (None if v is None else v.to(device)) for k, v in inp.items()}
 

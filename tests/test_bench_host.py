@@ -96,9 +96,16 @@ def test_roofline_arithmetic():
     assert abs(r["achieved"] - flops / 2e-3 / 1e12) < 1e-9 * r["achieved"]
     assert abs(r["frac"] - r["achieved"] / 1600.0) < 1e-12
     assert abs(r["frac_of_nominal"] - r["achieved"] / 2250.0) < 1e-12
-    # the power cap selects the sustained figure
-    capped = bench.roofline(mix, "mega_ffn", 2.0, peaks, "measured", {"reasons": ["sw_power_cap"]}, 8)
-    assert capped["peak"] == 1400.0 and "sustained" in capped["peak_kind"]
+    assert abs(r["frac_sustained"] - r["achieved"] / 1400.0) < 1e-12
+    # a timed region shorter than a second is compared with the burst figure
+    # even under the power cap; a capped region of a second or more with the
+    # sustained one
+    short = bench.roofline(mix, "mega_ffn", 2.0, peaks, "measured", {"reasons": ["sw_power_cap"]}, 8, region_s=0.05)
+    assert short["peak"] == 1600.0 and "burst" in short["peak_kind"]
+    long = bench.roofline(mix, "mega_ffn", 2.0, peaks, "measured", {"reasons": ["sw_power_cap"]}, 8, region_s=2.0)
+    assert long["peak"] == 1400.0 and "sustained" in long["peak_kind"]
+    uncapped = bench.roofline(mix, "mega_ffn", 2.0, peaks, "measured", {"reasons": []}, 8, region_s=2.0)
+    assert uncapped["peak"] == 1600.0
     # 64 rows per expert (gptoss): the touched experts' weight bytes bound it
     go = WORKLOADS["gptoss"]
     g = bench.roofline(go, "mega_ffn", 1.0, peaks, "measured", {"reasons": []}, 128)

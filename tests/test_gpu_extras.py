@@ -3,10 +3,11 @@ experts gated by the sink lanes (or ungated) -- against the fp64 oracle on
 seeded inputs; same bars as the core path."""
 import math
 
+import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import GpuRun, run_and_check_ex, to_dev
+from gpu_helpers import GpuRun, every_tile_tokens, oracle_route, run_and_check_ex, to_dev
 from mixture_experts_ffn_token_b200 import abi
 from mixture_experts_ffn_token_b200.workloads import WORKLOADS, make_inputs
 
@@ -75,9 +76,18 @@ def test_no_extras_equals_forward():
 
 
 @pytest.mark.parametrize("name", ["sink_shared", "mixtral_wfirst", "sink_masked", "mixtral_masked"])
-def test_extension_workloads_full_size_sampled(name):
-    import numpy as np
+def test_extension_workloads_full_size_every_tile(name):
+    """The extension workloads at full size: every token of the sink-shaped
+    ones; on the Mixtral-shaped ones the tokens whose rows reach every
+    128-row piece of every expert (masked tokens take no row, and the
+    masked rows must be exactly zero)."""
     wl = WORKLOADS[name] if name in WORKLOADS else WORKLOADS[name.split("_")[0]].replace(mask_frac=0.3)
-    rng = np.random.default_rng(7)
-    sample = np.unique(np.concatenate([[0, wl.num_tokens - 1], rng.choice(wl.num_tokens, 10, replace=False)]))
+    sample = None
+    if wl.name.startswith("mixtral"):
+        inp = make_inputs(wl, 0, device="cuda")
+        idx_ref, _, _ = oracle_route(wl, inp)
+        mask = None if inp["token_mask"] is None else inp["token_mask"].cpu().numpy()
+        sample = every_tile_tokens(idx_ref, wl.num_experts, token_mask=mask)
+        if mask is not None:  # some masked tokens too
+            sample = np.union1d(sample, np.flatnonzero(mask == 0)[:16])
     run_and_check_ex(wl, seed=0, device_inputs=True, sample_tokens=sample)

@@ -11,7 +11,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import FFN_TOL, GpuRun, check_weights, ffn_error, oracle_ffn, oracle_route, run_and_check, to_dev
+from gpu_helpers import (FFN_TOL, GpuRun, check_weights, every_tile_tokens, ffn_error, oracle_ffn, oracle_route,
+                         run_and_check, to_dev)
 from mixture_experts_ffn_token_b200 import abi
 from mixture_experts_ffn_token_b200.workloads import WORKLOADS, make_inputs
 
@@ -358,30 +359,61 @@ def test_zero_tokens():
 
 
 # ---------------------------------------------------------------- full size
-FULL_SAMPLE = 12
+# Every workload at full size in the benchmark's launch configuration (the
+# default single launch), in both tile orders: routing and weights for every
+# token; the layer output for every token where the oracle finishes in
+# seconds (tiny, gptoss, sink, decode: up to 464 GFLOP in fp64) and for
+# tokens whose rows reach every tile where it would take minutes (mixtral:
+# about 600 of 4096 tokens).
+FULL_EVERY_TOKEN = ("tiny", "gptoss", "sink", "decode")
 
 
-@pytest.mark.parametrize("name", ["mixtral", "gptoss", "sink", "decode"])
-def test_forward_full_size_sampled(name):
-    """Full-size workloads in the benchmark's launch configuration; routing and
-    CSR are compared for every token, the layer output on sampled tokens."""
+def full_size_reference(wl):
+    inp = make_inputs(wl, seed=0, device="cuda")
+    idx_ref, w_ref, s_ref = oracle_route(wl, inp)
+    tokens = None if wl.name in FULL_EVERY_TOKEN else every_tile_tokens(idx_ref, wl.num_experts)
+    ref = oracle_ffn(wl, inp, idx_ref, w_ref, tokens)
+    return inp, (idx_ref, w_ref, s_ref), tokens, ref
+
+
+def check_full_size_run(wl, inp, route_ref, tokens, ref):
+    idx_ref, w_ref, s_ref = route_ref
+    run = GpuRun(wl, inp, out_guard=64)
+    assert run.status == 0, f"device status {run.status:#x}"
+    assert np.array_equal(run.idx.cpu().numpy(), idx_ref)
+    check_weights(run.w.cpu().numpy(), w_ref)
+    if wl.num_sink > 0:
+        check_weights(run.sink.cpu().numpy(), s_ref)
+    got = run.out.float().cpu().numpy()
+    if tokens is not None:
+        got = got[tokens]
+    err = ffn_error(got, ref)
+    assert err <= FFN_TOL, f"ffn error {err:.3e} > {FFN_TOL}"
+    assert (run.out_full[wl.num_tokens * wl.hidden_dim:].float() == -7.0).all(), "output guard overwritten"
+    return err
+
+
+@pytest.mark.parametrize("name", ["tiny", "mixtral", "gptoss", "sink", "decode"])
+def test_forward_full_size_every_tile(name, monkeypatch):
+    """Both tile orders of the default single launch against one oracle
+    result: every 128-row piece of every expert has rows compared."""
     wl = WORKLOADS[name]
-    T = wl.num_tokens
-    rng = np.random.default_rng(123)
-    sample = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=min(T, FULL_SAMPLE), replace=False)]))
-    run_and_check(wl, seed=0, device_inputs=True, sample_tokens=sample)
+    inp, route_ref, tokens, ref = full_size_reference(wl)
+    if tokens is not None:
+        assert len(tokens) >= wl.num_experts and len(tokens) < wl.num_tokens
+    for order in ("static", "dynamic"):
+        monkeypatch.setenv("MOE_B200_TILE_SCHEDULE", order)
+        check_full_size_run(wl, inp, route_ref, tokens, ref)
 
 
 @pytest.mark.parametrize("name", ["mixtral", "sink"])
-def test_forward_full_size_sampled_cta_pair(name, monkeypatch):
+def test_forward_full_size_every_tile_cta_pair(name, monkeypatch):
     """The selectable CTA-pair variant at full size: 256-row pieces and
     M = 128 pair tails over every expert of the workload."""
     set_variant(monkeypatch, "two_launches_cta_pair")
     wl = WORKLOADS[name]
-    T = wl.num_tokens
-    rng = np.random.default_rng(124)
-    sample = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=min(T, FULL_SAMPLE), replace=False)]))
-    run_and_check(wl, seed=0, device_inputs=True, sample_tokens=sample)
+    inp, route_ref, tokens, ref = full_size_reference(wl)
+    check_full_size_run(wl, inp, route_ref, tokens, ref)
 
 
 @pytest.mark.parametrize("name,order", [("gptoss", "dynamic"), ("sink", "static"), ("sink", "dynamic")])
