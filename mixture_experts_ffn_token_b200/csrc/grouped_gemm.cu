@@ -120,6 +120,7 @@ struct GemmParams {
   int extra_arrivals;
   unsigned long long dep_timeout_ns;
   int a_direct;  // gate_up: A rows are rows within the expert's segment (A = x)
+  int k;         // routed slots per token (a slot's token is slot / k)
 };
 
 struct TileCoord {
@@ -416,13 +417,14 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoo
 // CTA walks the list in increasing order, so a down tile only ever waits on
 // gate_up tiles that precede it and that some resident CTA has already
 // started (the launch is cooperative: all CTAs are resident).
-template <int MODE, int PAIR, bool FUSED>
+template <int MODE, int PAIR, bool FUSED, bool GATHER>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                         const __grid_constant__ CUtensorMap mapA2, const __grid_constant__ CUtensorMap mapB2,
                         const __grid_constant__ CUtensorMap mapAh, const __grid_constant__ CUtensorMap mapA2h,
                         const GemmParams p, const GemmParams p2, int* arrivals, int* sched) {
   static_assert(!FUSED || (PAIR == 1 && MODE != MODE_DOWN), "the fused form is gate_up then down, one CTA a tile");
+  static_assert(!GATHER || (PAIR == 1 && MODE != MODE_DOWN), "rows are gathered for gate_up tiles of one CTA");
   using G = Geo<PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -537,25 +539,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const bool dyn = FUSED && sched != nullptr;  // dynamic tile order
 
   if (warp == 0) {
-    if (lane == 0) {
+    if (GATHER || lane == 0) {
       // ------------------------------------------------ TMA producer
+      // Lane 0 waits on the barriers, draws tiles and issues every copy.
+      // GATHER: the whole warp runs the loop, lane 0 still does all of the
+      // above, and for a gate_up tile each lane also issues one
+      // tile::gather4 per stage: the four rows 4*lane .. 4*lane+3 of the
+      // tile, read from x by the routing permutation (row -> slot -> token),
+      // into the same shared-memory image a 128-row box of the permuted copy
+      // would give.
+      auto bcast = [&](auto v) {
+        if constexpr (GATHER) return __shfl_sync(0xffffffffu, v, 0);
+        else return v;
+      };
       int it = 0;
       bool ok = true;
-      int t_next = dyn ? atomicAdd(sched, 1) : first_tile;
+      int t_next = first_tile;
+      if (dyn && lane == 0) t_next = atomicAdd(sched, 1);
+      t_next = bcast(t_next);
       for (int n = 0; ok; ++n) {
         const int t = t_next;
         if (dyn) {
           // hand tile number n to the consumers (the end marker too)
-          const int slot = n % kTileRing;
-          if (!mbar_wait(ring_empty0 + 8 * slot, (static_cast<uint32_t>(n / kTileRing) & 1u) ^ 1u, abort_flag,
-                         kTimeoutNs)) {
-            ok = false;
-            break;
+          bool stop = false;
+          if (lane == 0) {
+            const int slot = n % kTileRing;
+            if (!mbar_wait(ring_empty0 + 8 * slot, (static_cast<uint32_t>(n / kTileRing) & 1u) ^ 1u, abort_flag,
+                           kTimeoutNs)) {
+              ok = false;
+            } else {
+              s_ring[slot] = t;
+              mbar_arrive(ring_full0 + 8 * slot);
+              if (t >= total_tiles) stop = true;
+              else t_next = atomicAdd(sched, 1);  // in flight while this tile's copies are issued
+            }
           }
-          s_ring[slot] = t;
-          mbar_arrive(ring_full0 + 8 * slot);
-          if (t >= total_tiles) break;
-          t_next = atomicAdd(sched, 1);  // in flight while this tile's copies are issued
+          ok = bcast(ok);
+          stop = bcast(stop);
+          t_next = bcast(t_next);
+          if (!ok || stop) break;
         } else {
           if (t >= total_tiles) break;
           t_next = t + tile_stride;
@@ -573,18 +595,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t stage_tx = half ? G::STAGE_BYTES - HALF_A_BYTES : G::STAGE_BYTES;
         if constexpr (FUSED) {
           if (ph2) {
-            if (!wait_arrivals(arrivals + tc.piece, arrivals_needed, abort_flag, p.status, p.err_bit,
-                               p.dep_timeout_ns)) {
+            bool got = true;
+            if (lane == 0) {
+              got = wait_arrivals(arrivals + tc.piece, arrivals_needed, abort_flag, p.status, p.err_bit,
+                                  p.dep_timeout_ns);
+              if (got) fence_proxy_async_global();  // h stores (generic proxy) before the TMA reads of h
+            }
+            if (!bcast(got)) {
               ok = false;
               break;
             }
-            fence_proxy_async_global();  // h stores (generic proxy) before the TMA reads of h
+          }
+        }
+        // GATHER, gate_up tile: the tokens of this lane's four tile rows.
+        // Rows past the expert's segment (and slots outside [0, R), which the
+        // down epilogue flags) read the tile's first token; their results are
+        // discarded.
+        const bool gathered = GATHER && !ph2;
+        int tok[4] = {0, 0, 0, 0};
+        if constexpr (GATHER) {
+          if (gathered) {
+            const int s0 = p.perm[tc.row0];
+            const int first = s0 >= 0 && s0 < p.R ? s0 / p.k : 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int r = 4 * lane + j;
+              const int slot = r < tc.rows ? p.perm[tc.row0 + r] : -1;
+              tok[j] = slot >= 0 && slot < p.R ? slot / p.k : first;
+            }
           }
         }
         for (int kb = 0; kb < nkb; ++kb) {
           const int s = it % G::STAGES;
           const uint32_t ph = static_cast<uint32_t>(it / G::STAGES) & 1u;
-          if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kTimeoutNs)) {
+          bool got = true;
+          if (lane == 0) got = mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kTimeoutNs);
+          if (!bcast(got)) {
             ok = false;
             break;
           }
@@ -593,82 +639,108 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // the leader's full barrier counts both CTAs' bytes
           const uint32_t fb = PAIR == 2 ? map_to_rank(full0 + 8 * s, 0) : full0 + 8 * s;
           const int kc = kb * BK;
-          if (FUSED && ph2) {
-            // down tile: h rows of the piece, 256 columns of W_d
-            mbar_arrive_expect_tx(fb, stage_tx);
-            tma_load_2d(sa, half ? &mapA2h : &mapA2, fb, kc, arow);
-            if (p2.b_one_box) {
-              tma_load_4d(sb, &mapB2, fb, 0, kc, 4 * tc.n, tc.e);
-            } else {
-              const int c0 = tc.n * BN;
+          if (gathered) {
+            // 32 (or, for a half tile, 16) lanes each copy four rows of A
+            if (lane == 0) mbar_arrive_expect_tx(fb, stage_tx);
+            __syncwarp();
+            if (!half || lane < HALF_ROWS / 4)
+              tma_gather4(sa + static_cast<uint32_t>(lane) * 512u, &mapA, fb, kc, tok[0], tok[1], tok[2], tok[3]);
+            if (lane == 0) {
+              if (p.b_one_box) {
+                if constexpr (MODE == MODE_GATE_UP_CONCAT) tma_load_5d(sb, &mapB, fb, 0, kc, 2 * tc.n, 0, tc.e);
+                else tma_load_4d(sb, &mapB, fb, 0, kc, 4 * tc.n, tc.e);
+              } else if constexpr (MODE == MODE_GATE_UP_CONCAT) {
+                const int c0 = tc.n * 128;
+                tma_load_4d(sb, &mapB, fb, c0, 0, kc, tc.e);
+                tma_load_4d(sb + B_BOX_BYTES, &mapB, fb, c0 + 64, 0, kc, tc.e);
+                tma_load_4d(sb + 2 * B_BOX_BYTES, &mapB, fb, c0, 1, kc, tc.e);
+                tma_load_4d(sb + 3 * B_BOX_BYTES, &mapB, fb, c0 + 64, 1, kc, tc.e);
+              } else {
+                const int c0 = tc.n * BN;
 #pragma unroll
-              for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * B_BOX_BYTES, &mapB2, fb, c0 + 64 * j, kc, tc.e);
+                for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * B_BOX_BYTES, &mapB, fb, c0 + 64 * j, kc, tc.e);
+              }
             }
-          } else if (PAIR == 1 && p.b_one_box) {
-            // {64 columns, K, column block, (gate/up,) E} view: one copy lays
-            // the four 64-column boxes out exactly as four copies would
-            mbar_arrive_expect_tx(fb, stage_tx);
-            tma_load_2d(sa, half ? &mapAh : &mapA, fb, kc, arow);
-            if constexpr (MODE == MODE_GATE_UP_CONCAT) tma_load_5d(sb, &mapB, fb, 0, kc, 2 * tc.n, 0, tc.e);
-            else tma_load_4d(sb, &mapB, fb, 0, kc, 4 * tc.n, tc.e);
-          } else if constexpr (PAIR == 1) {
-            mbar_arrive_expect_tx(fb, stage_tx);
-            tma_load_2d(sa, half ? &mapAh : &mapA, fb, kc, arow);
-            if constexpr (MODE == MODE_GATE_UP_CONCAT) {
-              // 4-D view {D, 2 (gate/up), H, E}: two gate boxes then two up boxes.
-              const int c0 = tc.n * 128;
-              tma_load_4d(sb, &mapB, fb, c0, 0, kc, tc.e);
-              tma_load_4d(sb + B_BOX_BYTES, &mapB, fb, c0 + 64, 0, kc, tc.e);
-              tma_load_4d(sb + 2 * B_BOX_BYTES, &mapB, fb, c0, 1, kc, tc.e);
-              tma_load_4d(sb + 3 * B_BOX_BYTES, &mapB, fb, c0 + 64, 1, kc, tc.e);
-            } else {
-              // 3-D view {N, K, E}: four consecutive 64-column boxes.
-              const int c0 = tc.n * BN;
+          } else if (lane == 0) {
+            if (FUSED && ph2) {
+              // down tile: h rows of the piece, 256 columns of W_d
+              mbar_arrive_expect_tx(fb, stage_tx);
+              tma_load_2d(sa, half ? &mapA2h : &mapA2, fb, kc, arow);
+              if (p2.b_one_box) {
+                tma_load_4d(sb, &mapB2, fb, 0, kc, 4 * tc.n, tc.e);
+              } else {
+                const int c0 = tc.n * BN;
 #pragma unroll
-              for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * B_BOX_BYTES, &mapB, fb, c0 + 64 * j, kc, tc.e);
-            }
-          } else {
-            // The leader expects both CTAs' bytes on its own barrier; each
-            // CTA loads its rows of A (128, or 64 in a tail) and its half of
-            // the 256 columns.
-            if (leader) mbar_arrive_expect_tx(full0 + 8 * s, 2 * stage_tx);
-            tma_load_2d_pair(sa, half ? &mapAh : &mapA, fb, kc, arow);
-            if (p.b_one_box) {
-              // this CTA's two 64-column blocks in one copy (concatenated:
-              // the gate and the up block of h columns 64*rank .. +63 of the tile)
-              if constexpr (MODE == MODE_GATE_UP_CONCAT)
-                tma_load_5d_pair(sb, &mapB, fb, 0, kc, 2 * tc.n + static_cast<int>(rank), 0, tc.e);
-              else
-                tma_load_4d_pair(sb, &mapB, fb, 0, kc, 4 * tc.n + 2 * static_cast<int>(rank), tc.e);
-            } else if constexpr (MODE == MODE_GATE_UP_CONCAT) {
-              // the gate and the up block of h columns c0 .. c0+63
-              const int c0 = tc.n * 128 + 64 * static_cast<int>(rank);
-              tma_load_4d_pair(sb, &mapB, fb, c0, 0, kc, tc.e);
-              tma_load_4d_pair(sb + B_BOX_BYTES, &mapB, fb, c0, 1, kc, tc.e);
+                for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * B_BOX_BYTES, &mapB2, fb, c0 + 64 * j, kc, tc.e);
+              }
+            } else if (PAIR == 1 && p.b_one_box) {
+              // {64 columns, K, column block, (gate/up,) E} view: one copy lays
+              // the four 64-column boxes out exactly as four copies would
+              mbar_arrive_expect_tx(fb, stage_tx);
+              tma_load_2d(sa, half ? &mapAh : &mapA, fb, kc, arow);
+              if constexpr (MODE == MODE_GATE_UP_CONCAT) tma_load_5d(sb, &mapB, fb, 0, kc, 2 * tc.n, 0, tc.e);
+              else tma_load_4d(sb, &mapB, fb, 0, kc, 4 * tc.n, tc.e);
+            } else if constexpr (PAIR == 1) {
+              mbar_arrive_expect_tx(fb, stage_tx);
+              tma_load_2d(sa, half ? &mapAh : &mapA, fb, kc, arow);
+              if constexpr (MODE == MODE_GATE_UP_CONCAT) {
+                // 4-D view {D, 2 (gate/up), H, E}: two gate boxes then two up boxes.
+                const int c0 = tc.n * 128;
+                tma_load_4d(sb, &mapB, fb, c0, 0, kc, tc.e);
+                tma_load_4d(sb + B_BOX_BYTES, &mapB, fb, c0 + 64, 0, kc, tc.e);
+                tma_load_4d(sb + 2 * B_BOX_BYTES, &mapB, fb, c0, 1, kc, tc.e);
+                tma_load_4d(sb + 3 * B_BOX_BYTES, &mapB, fb, c0 + 64, 1, kc, tc.e);
+              } else {
+                // 3-D view {N, K, E}: four consecutive 64-column boxes.
+                const int c0 = tc.n * BN;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * B_BOX_BYTES, &mapB, fb, c0 + 64 * j, kc, tc.e);
+              }
             } else {
-              const int c0 = tc.n * BN + static_cast<int>(rank) * 128;
-              tma_load_3d_pair(sb, &mapB, fb, c0, kc, tc.e);
-              tma_load_3d_pair(sb + B_BOX_BYTES, &mapB, fb, c0 + 64, kc, tc.e);
+              // The leader expects both CTAs' bytes on its own barrier; each
+              // CTA loads its rows of A (128, or 64 in a tail) and its half of
+              // the 256 columns.
+              if (leader) mbar_arrive_expect_tx(full0 + 8 * s, 2 * stage_tx);
+              tma_load_2d_pair(sa, half ? &mapAh : &mapA, fb, kc, arow);
+              if (p.b_one_box) {
+                // this CTA's two 64-column blocks in one copy (concatenated:
+                // the gate and the up block of h columns 64*rank .. +63 of the tile)
+                if constexpr (MODE == MODE_GATE_UP_CONCAT)
+                  tma_load_5d_pair(sb, &mapB, fb, 0, kc, 2 * tc.n + static_cast<int>(rank), 0, tc.e);
+                else
+                  tma_load_4d_pair(sb, &mapB, fb, 0, kc, 4 * tc.n + 2 * static_cast<int>(rank), tc.e);
+              } else if constexpr (MODE == MODE_GATE_UP_CONCAT) {
+                // the gate and the up block of h columns c0 .. c0+63
+                const int c0 = tc.n * 128 + 64 * static_cast<int>(rank);
+                tma_load_4d_pair(sb, &mapB, fb, c0, 0, kc, tc.e);
+                tma_load_4d_pair(sb + B_BOX_BYTES, &mapB, fb, c0, 1, kc, tc.e);
+              } else {
+                const int c0 = tc.n * BN + static_cast<int>(rank) * 128;
+                tma_load_3d_pair(sb, &mapB, fb, c0, kc, tc.e);
+                tma_load_3d_pair(sb + B_BOX_BYTES, &mapB, fb, c0 + 64, kc, tc.e);
+              }
             }
           }
           ++it;
         }
       }
-      if (ok) {
-        // Tail: wait until the MMAs have released every stage, so that no
-        // tcgen05.commit arrival lands after this CTA exits.
-        for (int i = 0; i < G::STAGES; ++i, ++it) {
-          const int s = it % G::STAGES;
-          const uint32_t ph = static_cast<uint32_t>(it / G::STAGES) & 1u;
-          if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kTimeoutNs)) break;
-        }
-      } else if (leader) {
-        // Aborted: let the copies already issued land before shared memory
-        // is released (time-bounded, independent of the abort flag).
-        for (int s = 0; s < G::STAGES; ++s) {
-          if (it > s) {
-            const int last = s + ((it - 1 - s) / G::STAGES) * G::STAGES;
-            wait_time_only(full0 + 8 * s, static_cast<uint32_t>(last / G::STAGES) & 1u);
+      if (lane == 0) {
+        if (ok) {
+          // Tail: wait until the MMAs have released every stage, so that no
+          // tcgen05.commit arrival lands after this CTA exits.
+          for (int i = 0; i < G::STAGES; ++i, ++it) {
+            const int s = it % G::STAGES;
+            const uint32_t ph = static_cast<uint32_t>(it / G::STAGES) & 1u;
+            if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kTimeoutNs)) break;
+          }
+        } else if (leader) {
+          // Aborted: let the copies already issued land before shared memory
+          // is released (time-bounded, independent of the abort flag).
+          for (int s = 0; s < G::STAGES; ++s) {
+            if (it > s) {
+              const int last = s + ((it - 1 - s) / G::STAGES) * G::STAGES;
+              wait_time_only(full0 + 8 * s, static_cast<uint32_t>(last / G::STAGES) & 1u);
+            }
           }
         }
       }
@@ -859,7 +931,7 @@ int max_pair_clusters(size_t smem, int num_sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<MODE, 2, false>, &cfg) != cudaSuccess || n <= 0)
+  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<MODE, 2, false, false>, &cfg) != cudaSuccess || n <= 0)
     n = num_sms / 2;
   cached[dev] = n;
   return n;
@@ -872,6 +944,15 @@ int max_pair_clusters(size_t smem, int num_sms) {
 // MOE_B200_CTA_PAIR=2 selects the pair variant (1 forces the default).
 // One-copy B loads (default) or four 64-column copies per stage
 // (MOE_B200_B_ONE_BOX=0).
+// Row f1, the routed-row gather inside the gate_up GEMM
+// (MOE_B200_FUSED_GATHER=1): the producer warp's lanes copy the tile's rows
+// of x with tile::gather4 instead of a separate gather kernel writing the
+// permuted copy Xp.  Single-CTA tiles only.
+bool fused_gather_requested() {
+  const char* env = std::getenv("MOE_B200_FUSED_GATHER");
+  return env != nullptr && env[0] == '1';
+}
+
 bool one_box_enabled() {
   const char* env = std::getenv("MOE_B200_B_ONE_BOX");
   return !(env != nullptr && env[0] == '0');
@@ -884,19 +965,19 @@ int choose_pair(int /*R*/, int /*E*/) {
   return 1;
 }
 
-template <int MODE, int PAIR>
+template <int MODE, int PAIR, bool GATHER>
 cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const CUtensorMap& mapAh,
                         const GemmParams& p, int num_sms, cudaStream_t stream) {
   const int64_t max_pieces = p.R / Geo<PAIR>::PIECE + std::min(p.E, p.R);
   const int64_t max_tiles = max_pieces * p.n_tiles;
   const size_t smem = smem_bytes_for<PAIR>(p.E);
-  cudaError_t err = opt_in_dynamic_smem(reinterpret_cast<const void*>(grouped_gemm_kernel<MODE, PAIR, false>),
+  cudaError_t err = opt_in_dynamic_smem(reinterpret_cast<const void*>(grouped_gemm_kernel<MODE, PAIR, false, GATHER>),
                                         static_cast<int>(smem_bytes_for<PAIR>(kMaxExperts)));
   if (err != cudaSuccess) return err;
   if constexpr (PAIR == 1) {
     const int grid = static_cast<int>(std::min<int64_t>(max_tiles, num_sms));
-    grouped_gemm_kernel<MODE, 1, false><<<grid, NUM_THREADS, smem, stream>>>(mapA, mapB, mapA, mapB, mapAh, mapAh, p,
-                                                                              p, nullptr, nullptr);
+    grouped_gemm_kernel<MODE, 1, false, GATHER><<<grid, NUM_THREADS, smem, stream>>>(mapA, mapB, mapA, mapB, mapAh,
+                                                                                      mapAh, p, p, nullptr, nullptr);
     return cudaGetLastError();
   } else {
     const int clusters =
@@ -914,7 +995,8 @@ cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     // (the pair's tails of at most 128 rows copy 64 A rows per CTA through mapAh)
-    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 2, false>, mapA, mapB, mapA, mapB, mapAh, mapAh, p, p,
+    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 2, false, false>, mapA, mapB, mapA, mapB, mapAh, mapAh, p,
+                              p,
                               static_cast<int*>(nullptr), static_cast<int*>(nullptr));
   }
 }
@@ -960,7 +1042,14 @@ cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& ma
                     bool pair) {
   const bool down = MODE == MODE_DOWN;
   const int K = down ? a.D : a.H;
-  {
+  if (!down && a.gather) {
+    // rows of x gathered by token index: one-row boxes, four rows per tile::gather4
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(a.T)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {64, 1};
+    if (!encode_bf16_map(&mapA, a.A, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    mapAh = mapA;
+  } else {
     // with a_direct the A operand is x: T rows, indexed by the row within an expert
     const cuuint64_t rows = static_cast<cuuint64_t>(!down && a.a_direct ? a.T : a.R);
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), rows};
@@ -1005,6 +1094,7 @@ cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& ma
   }
   p.offsets = a.offsets;
   p.a_direct = !down && a.a_direct ? 1 : 0;
+  p.k = a.k;
   p.perm = a.perm;
   p.weights = a.weights;
   p.bias = a.bias;
@@ -1031,8 +1121,11 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t stream) {
   const int pair = choose_pair(a.R, a.E);
   cudaError_t err = prepare<MODE>(a, mapA, mapAh, mapB, p, pair == 2);
   if (err != cudaSuccess) return err;
-  if (pair == 2) return launch_with<MODE, 2>(mapA, mapB, mapAh, p, a.num_sms, stream);
-  return launch_with<MODE, 1>(mapA, mapB, mapAh, p, a.num_sms, stream);
+  if (pair == 2) return launch_with<MODE, 2, false>(mapA, mapB, mapAh, p, a.num_sms, stream);
+  if constexpr (MODE != MODE_DOWN) {
+    if (a.gather) return launch_with<MODE, 1, true>(mapA, mapB, mapAh, p, a.num_sms, stream);
+  }
+  return launch_with<MODE, 1, false>(mapA, mapB, mapAh, p, a.num_sms, stream);
 }
 
 // Rows per expert at which one bf16 weight byte carries as many FLOPs (2 per
@@ -1040,7 +1133,7 @@ cudaError_t launch_mode(const GroupedGemmArgs& a, cudaStream_t stream) {
 // (about 1.66 PFLOP/s over 6.5 TB/s).
 constexpr int64_t kRidgeRowsPerExpert = 256;
 
-template <int MODE>
+template <int MODE, bool GATHER>
 cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down, int* arrivals,
                          cudaStream_t stream) {
   if (up.R == 0) return cudaSuccess;
@@ -1055,7 +1148,7 @@ cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down,
   const int64_t max_pieces = p.R / BM + std::min(p.E, p.R);
   const int64_t max_tiles = max_pieces * (p.n_tiles + p2.n_tiles);
   const size_t smem = smem_bytes_for<1>(p.E);
-  err = opt_in_dynamic_smem(reinterpret_cast<const void*>(grouped_gemm_kernel<MODE, 1, true>),
+  err = opt_in_dynamic_smem(reinterpret_cast<const void*>(grouped_gemm_kernel<MODE, 1, true, GATHER>),
                             static_cast<int>(smem_bytes_for<1>(kMaxExperts)));
   if (err != cudaSuccess) return err;
   // Cooperative: the launch fails rather than run with CTAs that are not
@@ -1081,13 +1174,16 @@ cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down,
     if (env[0] == 's') dynamic = false;
   }
   int* sched = dynamic ? arrivals + mega_ffn_counters(up.R, up.E) - 1 : nullptr;
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 1, true>, mapA, mapB, mapA2, mapB2, mapAh, mapA2h, p, p2,
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 1, true, GATHER>, mapA, mapB, mapA2, mapB2, mapAh, mapA2h, p,
+                            p2,
                             arrivals, sched);
 }
 
 }  // namespace
 
 bool tensor_map_encoder_available() { return encoder() != nullptr; }
+
+bool fused_gather_enabled() { return fused_gather_requested() && choose_pair(0, 0) == 1; }
 
 cudaError_t launch_gemm_gate_up(const GroupedGemmArgs& a, cudaStream_t stream) {
   return a.gate_up_format == 0 ? launch_mode<MODE_GATE_UP_CONCAT>(a, stream)
@@ -1102,8 +1198,11 @@ int mega_ffn_counters(int R, int E) { return R / BM + std::min(E, R) + 1; }
 
 cudaError_t launch_mega_ffn(const GroupedGemmArgs& up, const GroupedGemmArgs& down, int* arrivals,
                             cudaStream_t stream) {
-  return up.gate_up_format == 0 ? launch_fused<MODE_GATE_UP_CONCAT>(up, down, arrivals, stream)
-                                : launch_fused<MODE_GATE_UP_INTERLEAVED>(up, down, arrivals, stream);
+  if (up.gather)
+    return up.gate_up_format == 0 ? launch_fused<MODE_GATE_UP_CONCAT, true>(up, down, arrivals, stream)
+                                  : launch_fused<MODE_GATE_UP_INTERLEAVED, true>(up, down, arrivals, stream);
+  return up.gate_up_format == 0 ? launch_fused<MODE_GATE_UP_CONCAT, false>(up, down, arrivals, stream)
+                                : launch_fused<MODE_GATE_UP_INTERLEAVED, false>(up, down, arrivals, stream);
 }
 
 }  // namespace moe

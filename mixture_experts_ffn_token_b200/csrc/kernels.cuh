@@ -105,6 +105,9 @@ struct GroupedGemmArgs {
   // gate_up only: A is x [T,H] itself and a slot's A row is its row within
   // its expert's segment (the shared experts' slots, token order per expert)
   int a_direct = 0;
+  // gate_up only: A is x [T,H] and the kernel gathers each tile's rows by the
+  // permutation itself (token = perm[p] / k); no Xp is read
+  int gather = 0;
   const __nv_bfloat16* W;   // [E,H,2D] (gate_up) or [E,D,H] (down)
   const __nv_bfloat16* bias;// [E,2D] / [E,H] or null
   __nv_bfloat16* out;       // h [R,D] (gate_up) or Y [R,H] slot rows (down)
@@ -127,5 +130,9 @@ cudaError_t launch_mega_ffn(const GroupedGemmArgs& up, const GroupedGemmArgs& do
 
 // Resolves cuTensorMapEncodeTiled through the runtime (no libcuda link).
 bool tensor_map_encoder_available();
+
+// Whether the gate_up GEMM gathers its rows of x itself in this process
+// (MOE_B200_FUSED_GATHER=1 with single-CTA tiles; off by default).
+bool fused_gather_enabled();
 
 }  // namespace moe

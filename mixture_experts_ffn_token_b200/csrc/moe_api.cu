@@ -262,8 +262,17 @@ moe_status_t enqueue_grouped_pass(const moe_config_t* c, int E, int k, int D, co
   const int T = c->num_tokens, H = c->hidden_dim;
   const int R = T * k;
   const bool fused = single_launch();
+  // row f1: the gate_up GEMM gathers its rows of x itself (not when the
+  // routing weight has to scale them first)
+  const bool gather_in_gemm = !a_direct && scale == nullptr && moe::fused_gather_enabled();
   rec(base);
-  if (!a_direct) {
+  if (gather_in_gemm) {
+    // no gather kernel to clear the single launch's counters
+    if (fused && R > 0 &&
+        cudaMemsetAsync(arr, 0, static_cast<size_t>(moe::mega_ffn_counters(R, E)) * sizeof(int), stream) !=
+            cudaSuccess)
+      return MOE_ERR_CUDA;
+  } else if (!a_direct) {
     const NvtxRange range("moe.gather");
     if (moe::launch_gather(static_cast<const __nv_bfloat16*>(x), perm, offsets, E, R, k, H, scale, xp, status,
                            num_sms, stream, fused ? arr : nullptr, fused ? moe::mega_ffn_counters(R, E) : 0) !=
@@ -286,8 +295,9 @@ moe_status_t enqueue_grouped_pass(const moe_config_t* c, int E, int k, int D, co
   g.limit = c->limit;
   g.status = status;
   g.num_sms = num_sms;
-  g.A = a_direct ? static_cast<const __nv_bfloat16*>(x) : xp;
+  g.A = (a_direct || gather_in_gemm) ? static_cast<const __nv_bfloat16*>(x) : xp;
   g.a_direct = a_direct ? 1 : 0;
+  g.gather = gather_in_gemm ? 1 : 0;
   g.W = static_cast<const __nv_bfloat16*>(gate_up_w);
   g.bias = static_cast<const __nv_bfloat16*>(gate_up_b);
   g.out = h;

@@ -48,7 +48,14 @@ VARIANTS = {"single_launch": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR"
             "single_launch_four_box": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1",
                                        "MOE_B200_B_ONE_BOX": "0"},
             "two_launches": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "1", "MOE_B200_B_ONE_BOX": "1"},
-            "two_launches_cta_pair": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "2"}}
+            "two_launches_cta_pair": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "2"},
+            # row f1: the gate_up GEMM gathers its rows of x itself (tile::gather4)
+            "single_launch_fused_gather": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1",
+                                           "MOE_B200_B_ONE_BOX": "1", "MOE_B200_FUSED_GATHER": "1"},
+            "single_launch_fused_gather_dynamic": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1",
+                                                   "MOE_B200_FUSED_GATHER": "1", "MOE_B200_TILE_SCHEDULE": "dynamic"},
+            "two_launches_fused_gather_four_box": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "1",
+                                                   "MOE_B200_B_ONE_BOX": "0", "MOE_B200_FUSED_GATHER": "1"}}
 
 
 def set_variant(monkeypatch, variant):
@@ -543,3 +550,36 @@ def test_no_writes_past_any_buffer(name, single_launch, monkeypatch):
     assert (idx_full[T * k:] == -12345).all() and (w_full[T * k:] == -3.0).all()
     assert (sink_full[T * S:] == -5.0).all()
     assert (out_full[T * H:] == -7.0).all()
+
+
+@pytest.mark.parametrize("order", ["static", "dynamic"])
+@pytest.mark.parametrize("name", sorted(SMALL) + sorted(ALIGNED))
+def test_fused_gather_equals_gather_kernel(name, order, monkeypatch):
+    """Row f1: the gate_up GEMM reading its rows of x by tile::gather4 gives
+    the same bits as the separate gather kernel followed by the GEMM (both
+    multiply the same bf16 rows), in one launch and in two."""
+    wl = {**SMALL, **ALIGNED}[name]
+    d = to_dev(make_inputs(wl, 31))
+    monkeypatch.setenv("MOE_B200_TILE_SCHEDULE", order)
+    for single in ("1", "0"):
+        monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", single)
+        monkeypatch.setenv("MOE_B200_FUSED_GATHER", "0")
+        ref = GpuRun(wl, d)
+        monkeypatch.setenv("MOE_B200_FUSED_GATHER", "1")
+        got = GpuRun(wl, d)
+        assert ref.status == 0 and got.status == 0
+        assert torch.equal(got.out, ref.out), (name, single)
+
+
+@pytest.mark.parametrize("name", ["mixtral", "sink", "gptoss"])
+def test_fused_gather_full_size_equals_gather_kernel(name, monkeypatch):
+    """Row f1 at full size in the single launch: bit-identical to the default
+    path, whose every tile is compared with the oracle above."""
+    wl = WORKLOADS[name]
+    d = to_dev(make_inputs(wl, 0, device="cuda"))
+    monkeypatch.setenv("MOE_B200_FUSED_GATHER", "0")
+    ref = GpuRun(wl, d)
+    monkeypatch.setenv("MOE_B200_FUSED_GATHER", "1")
+    got = GpuRun(wl, d)
+    assert ref.status == 0 and got.status == 0
+    assert torch.equal(got.out, ref.out)
