@@ -115,16 +115,30 @@ def max_over_ranks(x, dist_mod, device):
     return float(t.item())
 
 
-def launches_per_step(wl, single_launch):
-    """Kernels one call launches: router + 3-kernel CSR build (one kernel
-    when T*k <= 2048 and E <= 512), gather, the two grouped GEMMs (one
-    launch when fused), combine, and with shared experts their index and
-    GEMMs (plus their gather only when the router weight scales the input:
-    otherwise their gate_up GEMM reads x directly)."""
+def launches_per_step(wl, single_launch, csr_fused=False, fused_gather=False):
+    """Kernels one call launches: the router and the CSR build (one kernel
+    together when T*k <= 2048 and E <= 512; else the router plus one
+    cooperative CSR kernel when `csr_fused`, or plus count, scan and
+    scatter), the gather (none when the gate_up GEMM gathers its rows itself
+    and the router weight does not scale them), the two grouped GEMMs (one
+    launch when fused), the combine, and with shared experts their index
+    kernel and GEMMs (plus their gather only when the router weight scales
+    the input: otherwise their gate_up GEMM reads x directly)."""
     small = wl.num_tokens * wl.top_k <= 2048 and wl.num_experts <= 512
     gemms = 1 if single_launch else 2
     shared = (1 + (1 if wl.weight_first else 0) + gemms) if wl.num_shared > 0 else 0
-    return (1 if small else 4) + 1 + gemms + shared + 1
+    route_csr = 1 if small else (2 if csr_fused else 4)
+    gather = 0 if (fused_gather and not wl.weight_first) else 1
+    return route_csr + gather + gemms + shared + 1
+
+
+def csr_fused_active(wl, num_sms):
+    """Whether the library builds the CSR in one launch for this workload:
+    its chunks of 2048 slots fit on the GPU at once (MOE_B200_CSR_FUSED=0
+    turns it off)."""
+    if os.environ.get("MOE_B200_CSR_FUSED", "1").startswith("0"):
+        return False
+    return 0 < -(-wl.num_tokens * wl.top_k // 2048) <= num_sms
 
 
 def job_throughput(world, tokens_per_rank, ms_per_step):
@@ -644,8 +658,23 @@ def measure(args, wl, ctx, steps):
     out_bytes = T * H * 2
 
     # ---------------- host cost of one eager call (the public Python entry
-    # point and the library's enqueue work, no GPU wait)
+    # point and the library's enqueue work, no GPU wait), and of the
+    # library's C entry point alone (arguments marshalled once beforehand)
     host_us = host_enqueue_us(step, min(steps, 20), stream)
+    host_lib_us = None
+    if extras is None:
+        import ctypes
+        lib = abi.load_library()
+        p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+        c_args = (ctypes.byref(cfg), p(inp["x"]), p(inp["logits"]), p(inp["expert_bias"]), p(inp["global_scale"]),
+                p(inp["W_gu"]), p(inp["b_gu"]), p(inp["W_d"]), p(inp["b_d"]), p(out), p(idx), p(w), p(sink),
+                p(ws), ws.numel(), stream.cuda_stream)
+        fwd = lib.moe_forward
+
+        def c_step():
+            if fwd(*c_args) != 0:
+                raise RuntimeError("moe_forward failed")
+        host_lib_us = host_enqueue_us(c_step, min(steps, 20), stream)
 
     # ---------------- roofline of the dominant kernel, timed live by its event
     # pair in the timed region
@@ -656,6 +685,8 @@ def measure(args, wl, ctx, steps):
                   "shared_gemm_down": "(shared fused)"}.get(n, n) for n in names]
     flops = wl.flops()
     wbytes, used = touched_expert_bytes(wl, idx)
+    csr_fused = csr_fused_active(wl, torch.cuda.get_device_properties(local).multi_processor_count)
+    fused_gather = os.environ.get("MOE_B200_FUSED_GATHER", "0").startswith("1")
     dom_name = names[dom]
     clock_summary = clocks.summary()
     roof = roofline(wl, dom_name, kernel_ms, peaks, peak_kind, clock_summary, used, region_s=region_ms / 1e3)
@@ -677,7 +708,8 @@ def measure(args, wl, ctx, steps):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x_h_bytes,
                 "d2h_bytes_per_step": out_bytes},
         "host_us_per_call": host_us,
-        "gpu_launches": launches_per_step(wl, fused) * steps,
+        "host_us_per_call_c_abi": host_lib_us,
+        "gpu_launches": launches_per_step(wl, fused, csr_fused, fused_gather) * steps,
         "single_launch_ffn": fused,
         "clocks": clock_summary,
     }
@@ -691,7 +723,7 @@ PER_CONFIG = ("tiny", "gptoss", "sink", "decode")
 def compact(line):
     """The per-config entry: the figures of a full line that describe one workload."""
     keep = ("value", "unit", "ms_per_step", "steps", "tflops", "weight_gbs", "experts_touched", "roofline", "e2e",
-            "host_us_per_call", "gpu_launches", "clocks", "stages_ms")
+            "host_us_per_call", "host_us_per_call_c_abi", "gpu_launches", "clocks", "stages_ms")
     ent = {k: line[k] for k in keep}
     ent["workload"] = line["config"]["workload"]
     ent["l2"] = line["config"]["l2"]

@@ -75,6 +75,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return false;
 }
 
+// Acquire load at GPU scope (pairs with a release or a fence + atomic of
+// another CTA).
+__device__ __forceinline__ int ld_acquire_gpu(const int* addr) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+  return v;
+}
+
 // ---------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialization may begin while
 // its predecessor on the stream is still finishing.  griddep_wait() blocks

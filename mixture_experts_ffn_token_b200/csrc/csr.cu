@@ -175,6 +175,162 @@ __global__ void __launch_bounds__(kCsrThreads) csr_scatter_kernel(const int32_t*
   }
 }
 
+// The whole counting sort in ONE cooperative launch, one CTA per chunk of
+// kCsrChunk slots (used when the chunks fit on the GPU at once): each CTA
+// builds the per-warp histograms of its chunk and publishes the chunk's
+// counts; after a grid barrier every CTA reduces the (chunk x expert) count
+// table itself -- it is small -- to the expert offsets and its own chunk's
+// base positions, then places its slots exactly as csr_scatter_kernel does.
+// The result is bit-identical to the three-kernel form.  *barrier must be
+// zero at launch (the router kernel clears it, or the host); the wait is
+// bounded (timeout_ns, and an iteration cap) and records
+// MOE_DEVICE_ERR_TIMEOUT_CSR when it gives up, after which the CTA returns
+// without writing offsets or positions.
+constexpr uint64_t kCsrBarrierTimeoutNs = 1000000000ull;  // 1 s: far beyond any legitimate wait
+
+__global__ void __launch_bounds__(kCsrThreads) csr_fused_kernel(const int32_t* __restrict__ idx, int R, int E,
+                                                                int32_t* __restrict__ chunk_counts,
+                                                                int32_t* __restrict__ offsets,
+                                                                int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                                int* status, int* barrier,
+                                                                const uint8_t* __restrict__ mask, int k,
+                                                                int extra_arrivals, unsigned long long timeout_ns) {
+  griddep_wait();  // the previous kernel's results are complete and visible
+  extern __shared__ int sm[];
+  int* wcnt = sm;                  // [kCsrWarps][E]: per-warp counts, then their exclusive prefix over warps
+  int* cb = sm + kCsrWarps * E;    // [E]: this chunk's first position per expert
+  __shared__ int warp_tot[kCsrWarps];
+  __shared__ int s_go;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kCsrWarps * E; i += blockDim.x) wcnt[i] = 0;
+  __syncthreads();
+  const int64_t wbase = static_cast<int64_t>(blockIdx.x) * kCsrChunk + static_cast<int64_t>(warp) * kSlotsPerWarp;
+  int* my = wcnt + warp * E;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  constexpr int kRounds = kSlotsPerWarp / 32;
+  int ev[kRounds];
+  bool bad = false;
+#pragma unroll
+  for (int q = 0; q < kRounds; ++q) {
+    const int64_t s = wbase + 32 * q + lane;
+    int e = -1;
+    if (s < R && slot_live(mask, s, k)) {
+      e = idx[s];
+      if (e < 0 || e >= E) {
+        bad = true;
+        e = -1;
+      }
+    }
+    ev[q] = e;
+  }
+  if (bad) atomicOr(status, MOE_DEVICE_ERR_EXPERT_INDEX);
+  // per-warp histogram of the chunk
+#pragma unroll
+  for (int q = 0; q < kRounds; ++q) {
+    const int e = ev[q];
+    const uint32_t peers = __match_any_sync(0xffffffffu, e >= 0 ? e : E + lane);
+    if (e >= 0 && (peers & lt_mask) == 0) my[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // exclusive prefix over warps per expert; the chunk's count is the total
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < kCsrWarps; ++w) {
+      const int v = wcnt[w * E + e];
+      wcnt[w * E + e] = run;
+      run += v;
+    }
+    chunk_counts[static_cast<int64_t>(blockIdx.x) * E + e] = run;
+  }
+  __syncthreads();
+  // grid barrier: every chunk's counts are published before any CTA reads them
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(barrier, 1);
+    const int target = static_cast<int>(gridDim.x) + extra_arrivals;
+    bool ok = ld_acquire_gpu(barrier) >= target;
+    if (!ok) {
+      const uint64_t t0 = global_timer_ns();
+      for (uint32_t it = 1; it < (1u << 26) && !ok; ++it) {
+        __nanosleep(32);
+        ok = ld_acquire_gpu(barrier) >= target;
+        if (!ok && (it & 15u) == 0 && global_timer_ns() - t0 > timeout_ns) break;
+      }
+    }
+    if (!ok) atomicOr(status, MOE_DEVICE_ERR_TIMEOUT_CSR);
+    __threadfence();
+    s_go = ok ? 1 : 0;
+  }
+  __syncthreads();
+  if (!s_go) return;
+  // every CTA: per expert, the slots of earlier chunks and the total; an
+  // exclusive scan of the totals over experts gives the offsets (thread i
+  // owns experts 2i and 2i+1)
+  const int nchunks = static_cast<int>(gridDim.x);
+  const int e0 = 2 * threadIdx.x, e1 = e0 + 1;
+  int before0 = 0, before1 = 0, tot0 = 0, tot1 = 0;
+  for (int c = 0; c < nchunks; ++c) {
+    const int32_t* row = chunk_counts + static_cast<int64_t>(c) * E;
+    const int v0 = e0 < E ? row[e0] : 0;
+    const int v1 = e1 < E ? row[e1] : 0;
+    if (c < static_cast<int>(blockIdx.x)) {
+      before0 += v0;
+      before1 += v1;
+    }
+    tot0 += v0;
+    tot1 += v1;
+  }
+  const int local = tot0 + tot1;
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = lane < kCsrWarps ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += y;
+    }
+    if (lane < kCsrWarps) warp_tot[lane] = v;  // inclusive prefix of warp totals
+  }
+  __syncthreads();
+  const int excl = incl - local + (warp > 0 ? warp_tot[warp - 1] : 0);
+  if (e0 < E) {
+    cb[e0] = excl + before0;
+    if (blockIdx.x == 0) offsets[e0] = excl;
+  }
+  if (e1 < E) {
+    cb[e1] = excl + tot0 + before1;
+    if (blockIdx.x == 0) offsets[e1] = excl + tot0;
+  }
+  if (blockIdx.x == 0 && (e0 == E - 1 || e1 == E - 1)) offsets[E] = excl + local;
+  __syncthreads();
+  griddep_launch_dependents();
+  // positions in slot order (as csr_scatter_kernel)
+#pragma unroll
+  for (int q = 0; q < kRounds; ++q) {
+    const int64_t s = wbase + 32 * q + lane;
+    const int e = ev[q];
+    const uint32_t peers = __match_any_sync(0xffffffffu, e >= 0 ? e : E + lane);
+    int base = 0;
+    if (e >= 0) base = cb[e] + my[e];
+    __syncwarp();
+    if (e >= 0) {
+      const int pos = base + __popc(peers & lt_mask);
+      perm[pos] = static_cast<int32_t>(s);
+      if (inv != nullptr) inv[s] = pos;
+      if ((peers & lt_mask) == 0) my[e] += __popc(peers);
+    }
+    __syncwarp();
+  }
+}
+
 }  // namespace
 
 bool pdl_enabled() {
@@ -366,6 +522,55 @@ cudaError_t launch_csr_scatter(const int32_t* idx, int R, int E, const int32_t* 
   }
   return launch_pdl(csr_scatter_kernel, dim3(nchunks), dim3(kCsrThreads), smem, stream, idx, R, E, chunk_base, perm,
                     inv, mask, k);
+}
+
+bool csr_fused_enabled(int R, int num_sms) {
+  const char* env = std::getenv("MOE_B200_CSR_FUSED");
+  if (env != nullptr && env[0] == '0') return false;
+  const int n = csr_num_chunks(R);
+  return n > 0 && n <= num_sms;
+}
+
+cudaError_t launch_csr_fused(const int32_t* idx, int R, int E, int32_t* chunk_counts, int32_t* offsets, int32_t* perm,
+                             int32_t* inv, int* status, int* barrier, const uint8_t* mask, int k,
+                             cudaStream_t stream) {
+  const int nchunks = csr_num_chunks(R);
+  if (nchunks == 0) return cudaSuccess;
+  const size_t smem = (static_cast<size_t>(kCsrWarps) + 1) * E * sizeof(int);
+  if (smem > 48 * 1024) {
+    // once per device, for the largest expert count
+    cudaError_t err = opt_in_dynamic_smem(reinterpret_cast<const void*>(csr_fused_kernel),
+                                          static_cast<int>((static_cast<size_t>(kCsrWarps) + 1) * kMaxExperts *
+                                                           sizeof(int)));
+    if (err != cudaSuccess) return err;
+  }
+  // cooperative: the launch fails rather than run CTAs that are not all
+  // resident, which the grid barrier needs
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(nchunks));
+  cfg.blockDim = dim3(kCsrThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // Test hook for the bounded grid barrier: MOE_B200_TEST_STALL_CSR_MS=<ms>
+  // makes every CTA wait for one arrival more than will ever come, giving
+  // up after <ms>; the launch then records MOE_DEVICE_ERR_TIMEOUT_CSR and
+  // ends normally.
+  int extra = 0;
+  unsigned long long timeout_ns = kCsrBarrierTimeoutNs;
+  if (const char* env = std::getenv("MOE_B200_TEST_STALL_CSR_MS")) {
+    const long ms = std::strtol(env, nullptr, 10);
+    if (ms > 0) {
+      extra = 1;
+      timeout_ns = static_cast<unsigned long long>(std::min(ms, 1000L)) * 1000000ull;
+    }
+  }
+  return cudaLaunchKernelEx(&cfg, csr_fused_kernel, idx, R, E, chunk_counts, offsets, perm, inv, status, barrier, mask,
+                            k, extra, timeout_ns);
 }
 
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, const int32_t* offsets, int E, int R, int k,

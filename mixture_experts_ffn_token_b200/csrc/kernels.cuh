@@ -49,7 +49,7 @@ struct RouterArgs {
   int32_t* idx;              // [T,k]
   float* w;                  // [T,k]
   float* sink_w;             // [T,S] or null
-  int* status_reset;         // zeroed by the first thread, or null
+  int* status_reset;         // status_reset[0] (status) and [1] (CSR grid barrier) zeroed by the first thread, or null
 };
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t stream);
 
@@ -72,6 +72,13 @@ cudaError_t launch_csr_scan(const int32_t* chunk_counts, int nchunks, int E, int
                             int32_t* offsets, cudaStream_t stream);
 cudaError_t launch_csr_scatter(const int32_t* idx, int R, int E, const int32_t* chunk_base, int32_t* perm,
                                int32_t* inv, const uint8_t* mask, int k, cudaStream_t stream);
+// The three CSR kernels as one cooperative launch (one CTA per chunk), used
+// when the chunks fit on the GPU at once (csr_num_chunks(R) <= num_sms) unless
+// MOE_B200_CSR_FUSED=0; *barrier must be zero at launch.
+bool csr_fused_enabled(int R, int num_sms);
+cudaError_t launch_csr_fused(const int32_t* idx, int R, int E, int32_t* chunk_counts, int32_t* offsets, int32_t* perm,
+                             int32_t* inv, int* status, int* barrier, const uint8_t* mask, int k,
+                             cudaStream_t stream);
 // shared slots: offsets[i] = i*T, perm[i*T + t] = t*Ns + i; also clears
 // zero[0 .. n_zero) (may be null / 0).
 cudaError_t launch_shared_index(int T, int Ns, int32_t* offsets, int32_t* perm, int num_sms, cudaStream_t stream,

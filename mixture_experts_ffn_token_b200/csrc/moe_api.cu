@@ -354,16 +354,31 @@ moe_status_t enqueue_ffn(const moe_config_t* c, const void* x, const void* gate_
   return MOE_OK;
 }
 
+// The CSR build: one cooperative launch when the chunks fit on the GPU at
+// once, else count -> scan -> scatter.  The workspace's second int (right
+// after the status word) is the one-launch form's grid barrier and must be
+// zero here (the router clears both, or the caller's memset).
 moe_status_t enqueue_csr(const moe_config_t* c, const int32_t* idx, int32_t* offsets, int32_t* perm, int32_t* inv,
-                         void* ws, const WsLayout& L, cudaStream_t stream, cudaEvent_t const* ev,
+                         void* ws, const WsLayout& L, int num_sms, cudaStream_t stream, cudaEvent_t const* ev,
                          const uint8_t* mask = nullptr) {
   const int R = c->num_tokens * c->top_k, E = c->num_experts, k = c->top_k;
   const Recorder rec{ev, stream};
+  int* status = at<int>(ws, L.status);
   rec(0);
+  if (moe::csr_fused_enabled(R, num_sms)) {
+    {
+      const NvtxRange range("moe.csr_fused");
+      if (moe::launch_csr_fused(idx, R, E, at<int32_t>(ws, L.chunk_counts), offsets, perm, inv, status, status + 1,
+                                mask, k, stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    rec(1);
+    rec(2);
+    return MOE_OK;
+  }
   {
     const NvtxRange range("moe.csr_count");
-    if (moe::launch_csr_count(idx, R, E, at<int32_t>(ws, L.chunk_counts), at<int>(ws, L.status), mask, k, stream) !=
-        cudaSuccess)
+    if (moe::launch_csr_count(idx, R, E, at<int32_t>(ws, L.chunk_counts), status, mask, k, stream) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
   rec(1);
@@ -463,7 +478,7 @@ moe_status_t forward_impl(const moe_config_t* cfg, const moe_extras_t* extras, c
       const NvtxRange range("moe.router");
       if (moe::launch_router(ra, stream) != cudaSuccess) return MOE_ERR_CUDA;
     }
-    if ((st = enqueue_csr(cfg, idx, offsets, perm, nullptr, ws, L, stream, ev != nullptr ? ev + 1 : nullptr,
+    if ((st = enqueue_csr(cfg, idx, offsets, perm, nullptr, ws, L, num_sms, stream, ev != nullptr ? ev + 1 : nullptr,
                           ex.mask)) != MOE_OK)
       return st;
   }
@@ -577,8 +592,9 @@ moe_status_t moe_create_indices(const moe_config_t* cfg, const int32_t* expert_i
   int num_sms = 0;
   if ((st = current_device(&num_sms)) != MOE_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
-  return enqueue_csr(cfg, expert_indices, expert_offsets, permutation, inverse, workspace, L, s, nullptr);
+  // the status word and the CSR build's grid barrier start at zero
+  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, 2 * sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+  return enqueue_csr(cfg, expert_indices, expert_offsets, permutation, inverse, workspace, L, num_sms, s, nullptr);
 }
 
 moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x, const void* gate_up_w, const void* gate_up_b,
@@ -655,7 +671,8 @@ moe_status_t moe_device_status(const void* workspace, int32_t* device_status, mo
   if (cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
   *device_status = v;
-  if (v & (MOE_DEVICE_ERR_TIMEOUT_GEMM1 | MOE_DEVICE_ERR_TIMEOUT_GEMM2)) return MOE_ERR_DEVICE_TIMEOUT;
+  if (v & (MOE_DEVICE_ERR_TIMEOUT_GEMM1 | MOE_DEVICE_ERR_TIMEOUT_GEMM2 | MOE_DEVICE_ERR_TIMEOUT_CSR))
+    return MOE_ERR_DEVICE_TIMEOUT;
   return MOE_OK;
 }
 
@@ -719,7 +736,7 @@ extern "C" moe_status_t moe_create_indices_noalloc(const moe_config_t* cfg, cons
   L.chunk_base = kNoAllocHeaderBytes + kNoAllocMaxCells * sizeof(int32_t);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // The histogram and base tables are fully rewritten by every call; only the
-  // status word has to start at zero.
-  if (cudaMemsetAsync(base, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
-  return enqueue_csr(cfg, expert_indices, expert_offsets, permutation, inverse, base, L, s, nullptr);
+  // status word and the grid barrier word after it have to start at zero.
+  if (cudaMemsetAsync(base, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  return enqueue_csr(cfg, expert_indices, expert_offsets, permutation, inverse, base, L, num_sms, s, nullptr);
 }

@@ -130,7 +130,10 @@ template <int NPL, bool SINK, bool BF16>
 __global__ void __launch_bounds__(128) router_kernel(const RouterArgs a) {
   griddep_wait();  // the previous kernel's results are complete and visible
   griddep_launch_dependents();
-  if (a.status_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.status_reset = 0;
+  if (a.status_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+    a.status_reset[0] = 0;  // device status word
+    a.status_reset[1] = 0;  // grid barrier of the one-launch CSR build that follows
+  }
   const int lane = threadIdx.x & 31;
   const int t = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
   if (t >= a.T) return;

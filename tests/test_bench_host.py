@@ -115,3 +115,22 @@ def test_roofline_arithmetic():
     # the gate_up GEMM alone (two launches): 4 R H D FLOPs
     up = bench.roofline(mix, "gemm_gate_up", 1.0, peaks, "measured", {"reasons": []}, 8)
     assert abs(up["achieved"] - 4 * 8192 * 4096 * 14336 / 1e-3 / 1e12) < 1e-9 * up["achieved"]
+
+
+def test_launches_per_step():
+    from mixture_experts_ffn_token_b200.workloads import WORKLOADS
+    W = WORKLOADS
+    # small problems: route+CSR in one kernel, gather, single-launch FFN, combine
+    assert bench.launches_per_step(W["tiny"], True) == 4
+    assert bench.launches_per_step(W["decode"], True, csr_fused=True) == 4
+    # router + one CSR kernel + gather + FFN + combine
+    assert bench.launches_per_step(W["sink"], True, csr_fused=True) == 5
+    assert bench.launches_per_step(W["sink"], True, csr_fused=False) == 7
+    assert bench.launches_per_step(W["sink"], False, csr_fused=False) == 8
+    # the gate_up GEMM gathering its own rows drops the gather kernel
+    assert bench.launches_per_step(W["mixtral"], True, csr_fused=True, fused_gather=True) == 4
+    # ... unless the router weight scales the rows first
+    assert bench.launches_per_step(W["mixtral_wfirst"], True, csr_fused=True, fused_gather=True) == 5
+    # shared experts reading x directly: index kernel + single launch
+    assert bench.launches_per_step(W["sink_shared"], True, csr_fused=True) == 7
+    assert bench.csr_fused_active(W["sink"], 148) and not bench.csr_fused_active(W["sink"], 16)

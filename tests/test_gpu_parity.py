@@ -267,8 +267,14 @@ def test_sink_router_extremes():
     assert torch.allclose(tot.cpu(), torch.full((64,), 2.5 * 0.75, dtype=torch.float64), rtol=1e-6)
 
 
-@pytest.mark.parametrize("T,E,k", [(1, 1, 1), (1000, 16, 4), (4096, 128, 6), (7, 1024, 3), (50000, 8, 2)])
-def test_create_indices(T, E, k):
+@pytest.mark.parametrize("fused", ["1", "0"])
+@pytest.mark.parametrize("T,E,k", [(1, 1, 1), (1000, 16, 4), (4096, 128, 6), (7, 1024, 3), (50000, 8, 2),
+                                   (8192, 1024, 6), (160000, 64, 2)])
+def test_create_indices(T, E, k, fused, monkeypatch):
+    """Both forms of the CSR build (one cooperative launch, or count -> scan
+    -> scatter) against the oracle's counting sort, bit for bit.  160000 x 2
+    slots are more chunks than SMs, so that case always takes three launches."""
+    monkeypatch.setenv("MOE_B200_CSR_FUSED", fused)
     g = torch.Generator().manual_seed(T + E)
     idx = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32) if T < 5000 else \
         torch.argsort(torch.rand(T, E, generator=g), dim=1)[:, :k].to(torch.int32)
@@ -286,7 +292,9 @@ def test_create_indices(T, E, k):
     assert abi.moe_device_status(ws) == 0
 
 
-def test_create_indices_flags_bad_expert():
+@pytest.mark.parametrize("fused", ["1", "0"])
+def test_create_indices_flags_bad_expert(fused, monkeypatch):
+    monkeypatch.setenv("MOE_B200_CSR_FUSED", fused)
     wl = WORKLOADS["tiny"].replace(num_tokens=10, num_experts=8, top_k=2)
     cfg = abi.make_config(wl)
     idx = torch.randint(0, 8, (10, 2), dtype=torch.int32)
@@ -583,3 +591,17 @@ def test_fused_gather_full_size_equals_gather_kernel(name, monkeypatch):
     got = GpuRun(wl, d)
     assert ref.status == 0 and got.status == 0
     assert torch.equal(got.out, ref.out)
+
+
+@pytest.mark.parametrize("name", ["sink", "mixtral", "gptoss"])
+def test_csr_forms_give_the_same_forward(name, monkeypatch):
+    """The full-size forward with the one-launch CSR build (default) and with
+    three launches: identical routing, permutation and output bits."""
+    wl = WORKLOADS[name]
+    d = to_dev(make_inputs(wl, 3, device="cuda"))
+    monkeypatch.setenv("MOE_B200_CSR_FUSED", "1")
+    a = GpuRun(wl, d)
+    monkeypatch.setenv("MOE_B200_CSR_FUSED", "0")
+    b = GpuRun(wl, d)
+    assert a.status == 0 and b.status == 0
+    assert torch.equal(a.out, b.out) and torch.equal(a.idx, b.idx)

@@ -41,3 +41,35 @@ def test_down_tile_wait_gives_up_and_recovers(wl, order, monkeypatch):
     # the context is intact: the same call without the hook is correct again
     monkeypatch.delenv("MOE_B200_TEST_STALL_DOWN_TILES_MS")
     run_and_check(wl, seed=21)
+
+
+def test_csr_grid_barrier_gives_up_and_recovers(monkeypatch):
+    """The one-launch CSR build waits at a grid barrier for every chunk's
+    counts; with one arrival more requested than any launch delivers, every
+    CTA gives up after the hook's limit, records MOE_DEVICE_ERR_TIMEOUT_CSR
+    and returns; the next call, without the hook, matches the oracle."""
+    import numpy as np
+
+    import oracle
+    T, E, k = 8192, 128, 6
+    wl = WORKLOADS["tiny"].replace(num_tokens=T, num_experts=E, top_k=k)
+    cfg = abi.make_config(wl)
+    g = torch.Generator().manual_seed(5)
+    idx = torch.argsort(torch.rand(T, E, generator=g), dim=1)[:, :k].to(torch.int32).cuda()
+    ws = torch.empty(abi.moe_workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    monkeypatch.setenv("MOE_B200_CSR_FUSED", "1")
+    monkeypatch.setenv("MOE_B200_TEST_STALL_CSR_MS", "20")
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    abi.moe_create_indices(cfg, idx, off, perm, None, ws)
+    stop.record()
+    torch.cuda.synchronize()
+    assert abi.moe_device_status(ws) & abi.DEVICE_ERR_TIMEOUT_CSR
+    assert start.elapsed_time(stop) < 1000.0
+    monkeypatch.delenv("MOE_B200_TEST_STALL_CSR_MS")
+    abi.moe_create_indices(cfg, idx, off, perm, None, ws)
+    assert abi.moe_device_status(ws) == 0
+    _, o_ref, p_ref, _ = oracle.create_indices(idx.cpu().numpy(), E)
+    assert np.array_equal(off.cpu().numpy(), o_ref) and np.array_equal(perm.cpu().numpy(), p_ref)
