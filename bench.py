@@ -416,26 +416,45 @@ def timed_steps(step, steps, stream, flush):
 def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None, copy_streams=1, steps=None):
     """K steps of moe_forward (moe_forward_ex when `make_ex` builds its extras
     from a device token mask) fed from, and returning to, pinned host memory.
-    The token mask, when there is one, is a per-step input and is copied too.
-    Each per-step copy is split by rows over `copy_streams` streams per
-    direction (so that several copy engines share it), double-buffered so
-    that step i's copies overlap the compute of its neighbours.
-    Returns the device time (max over ranks) of the whole region in ms."""
+    Each step's inputs -- x, the logits and, when there is one, the token
+    mask -- sit back to back in one pinned staging buffer and cross to the
+    device in one copy (split by bytes over `copy_streams` streams, so that
+    several copy engines can share it); its output comes back in one copy
+    (split by rows).  Double-buffered, so that step i's copies overlap the
+    compute of its neighbours.  Returns (device time of the whole region in
+    ms, max over ranks; host->device bytes per step)."""
     T, H = inp["x"].shape
-    x_h = inp["x"].cpu().pin_memory()
-    lg_h = inp["logits"].cpu().pin_memory()
     has_mask = inp["token_mask"] is not None
-    mask_h = inp["token_mask"].cpu().pin_memory() if has_mask else None
-    mask_d = [torch.empty_like(inp["token_mask"]) if has_mask else None for _ in range(2)]
+    parts = [inp["x"], inp["logits"]] + ([inp["token_mask"]] if has_mask else [])
+    offs, size = [], 0
+    for t in parts:
+        offs.append(size)
+        size += (t.numel() * t.element_size() + 255) // 256 * 256
+    stage_h = torch.zeros(size, dtype=torch.uint8).pin_memory()
+    for t, o in zip(parts, offs):
+        nb = t.numel() * t.element_size()
+        stage_h[o:o + nb].copy_(t.detach().cpu().contiguous().view(-1).view(torch.uint8))
+    stage_d = [torch.empty(size, dtype=torch.uint8, device="cuda") for _ in range(2)]
+
+    def view(buf, i):
+        t, o = parts[i], offs[i]
+        return buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+
+    x_d = [view(stage_d[b], 0) for b in range(2)]
+    lg_d = [view(stage_d[b], 1) for b in range(2)]
+    mask_d = [view(stage_d[b], 2) if has_mask else None for b in range(2)]
     ex_b = [make_ex(mask_d[b]) if make_ex is not None else None for b in range(2)]
     out_h = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    x_d = [torch.empty_like(inp["x"]) for _ in range(2)]
-    lg_d = [torch.empty_like(inp["logits"]) for _ in range(2)]
     out_d = [torch.empty((T, H), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    # the layer call for each buffer set, marshalled once (abi.BoundForward
+    # still runs the whole C entry point every call)
+    calls = [abi.BoundForward(cfg, x_d[b], lg_d[b], inp["W_gu"], inp["W_d"], out_d[b], ws, extras=ex_b[b],
+                              stream=stream, **kw) for b in range(2)]
     n = max(1, min(copy_streams, T))
     h2d = [torch.cuda.Stream() for _ in range(n)]
     d2h = [torch.cuda.Stream() for _ in range(n)]
-    cut = [T * q // n for q in range(n + 1)]  # row ranges of the split copies
+    bcut = [size * q // n // 256 * 256 for q in range(n)] + [size]  # byte ranges of the split input copy
+    cut = [T * q // n for q in range(n + 1)]                         # row ranges of the split output copy
 
     def region(steps):
         in_ready = [[torch.cuda.Event() for _ in range(n)] for _ in range(steps)]
@@ -448,25 +467,18 @@ def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None, copy_streams=1, 
         for i in range(steps):
             b = i % 2
             for q, st in enumerate(h2d):
-                lo, hi = cut[q], cut[q + 1]
+                lo, hi = bcut[q], bcut[q + 1]
                 with torch.cuda.stream(st):
                     if i >= 2:
                         st.wait_event(fwd_done[i - 2])      # buffer b no longer read by step i-2
-                    x_d[b][lo:hi].copy_(x_h[lo:hi], non_blocking=True)
-                    lg_d[b][lo:hi].copy_(lg_h[lo:hi], non_blocking=True)
-                    if has_mask:
-                        mask_d[b][lo:hi].copy_(mask_h[lo:hi], non_blocking=True)
+                    stage_d[b][lo:hi].copy_(stage_h[lo:hi], non_blocking=True)
                     in_ready[i][q].record(st)
             for ev in in_ready[i]:
                 stream.wait_event(ev)
             if i >= 2:
                 for ev in out_done[i - 2]:
                     stream.wait_event(ev)                   # out_d[b] copied out by step i-2
-            if ex_b[b] is None:
-                abi.moe_forward(cfg, x_d[b], lg_d[b], inp["W_gu"], inp["W_d"], out_d[b], ws, stream=stream, **kw)
-            else:
-                abi.moe_forward_ex(cfg, ex_b[b], x_d[b], lg_d[b], inp["W_gu"], inp["W_d"], out_d[b], ws,
-                                   stream=stream, **kw)
+            calls[b]()
             fwd_done[i].record(stream)
             for q, st in enumerate(d2h):
                 lo, hi = cut[q], cut[q + 1]
@@ -489,7 +501,7 @@ def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None, copy_streams=1, 
     ms = region(steps)
     if not torch.equal(out_h[(steps - 1) % 2], out_d[(steps - 1) % 2].cpu()):
         raise RuntimeError("e2e: host copy of the output differs from the device result")
-    return max_over_ranks(ms, dist, "cuda")
+    return max_over_ranks(ms, dist, "cuda"), size
 
 
 def host_enqueue_us(step, calls, stream):
@@ -650,11 +662,9 @@ def measure(args, wl, ctx, steps):
     # from pinned memory and its output device->host inside the timed region.
     # Copies run on their own streams, double-buffered, so step i's copies
     # overlap the compute of its neighbours.
-    e2e_ms = run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex, copy_streams=args.copy_streams, steps=steps)
+    e2e_ms, x_h_bytes = run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex, copy_streams=args.copy_streams,
+                                steps=steps)
     e2e_value = job_throughput(world, T, e2e_ms / steps)
-    x_h_bytes = inp["x"].numel() * 2 + inp["logits"].numel() * 4
-    if inp["token_mask"] is not None:
-        x_h_bytes += inp["token_mask"].numel()
     out_bytes = T * H * 2
 
     # ---------------- host cost of one eager call (the public Python entry

@@ -238,6 +238,36 @@ def moe_forward(cfg, x, logits, gate_up_w, down_w, out, workspace, gate_up_b=Non
                                       _p(workspace), workspace.numel(), _stream(stream)), "moe_forward")
 
 
+class BoundForward:
+    """moe_forward (or, with `extras`, moe_forward_ex) bound to fixed tensors
+    and a stream: the argument marshalling happens once, and each call()
+    runs the C entry point itself -- validation, workspace checks and every
+    kernel launch happen on every call, as with moe_forward.  The object
+    keeps its tensors alive; bind again for other buffers or another
+    stream."""
+
+    def __init__(self, cfg, x, logits, gate_up_w, down_w, out, workspace, gate_up_b=None, down_b=None,
+                 expert_bias=None, global_scale=None, expert_indices_out=None, expert_weights_out=None,
+                 sink_weights_out=None, extras=None, stream=None):
+        lib = load_library()
+        self._keep = (cfg, x, logits, gate_up_w, down_w, out, workspace, gate_up_b, down_b, expert_bias,
+                      global_scale, expert_indices_out, expert_weights_out, sink_weights_out, extras)
+        common = (_p(x), _p(logits), _p(expert_bias), _p(global_scale), _p(gate_up_w), _p(gate_up_b), _p(down_w),
+                  _p(down_b), _p(out), _p(expert_indices_out), _p(expert_weights_out), _p(sink_weights_out),
+                  _p(workspace), workspace.numel(), _stream(stream))
+        if extras is None:
+            self._fn, self._where = lib.moe_forward, "moe_forward"
+            self._args = (ctypes.byref(cfg),) + common
+        else:
+            self._fn, self._where = lib.moe_forward_ex, "moe_forward_ex"
+            self._args = (ctypes.byref(cfg), ctypes.byref(extras)) + common + (None,)
+
+    def __call__(self):
+        st = self._fn(*self._args)
+        if st != MOE_OK:
+            raise MoEError(st, self._where)
+
+
 def _event_handles(events, stream):
     """cudaEvent_t handles of torch.cuda.Event objects (None stays NULL)."""
     handles = []

@@ -333,10 +333,7 @@ __global__ void __launch_bounds__(kCsrThreads) csr_fused_kernel(const int32_t* _
 
 }  // namespace
 
-bool pdl_enabled() {
-  const char* env = std::getenv("MOE_B200_PDL");
-  return !(env != nullptr && env[0] == '0');
-}
+bool pdl_enabled() { return switches().pdl; }
 
 cudaError_t opt_in_dynamic_smem(const void* func, int bytes) {
   struct Done {
@@ -525,8 +522,7 @@ cudaError_t launch_csr_scatter(const int32_t* idx, int R, int E, const int32_t* 
 }
 
 bool csr_fused_enabled(int R, int num_sms) {
-  const char* env = std::getenv("MOE_B200_CSR_FUSED");
-  if (env != nullptr && env[0] == '0') return false;
+  if (!switches().csr_fused) return false;
   const int n = csr_num_chunks(R);
   return n > 0 && n <= num_sms;
 }
@@ -562,12 +558,9 @@ cudaError_t launch_csr_fused(const int32_t* idx, int R, int E, int32_t* chunk_co
   // ends normally.
   int extra = 0;
   unsigned long long timeout_ns = kCsrBarrierTimeoutNs;
-  if (const char* env = std::getenv("MOE_B200_TEST_STALL_CSR_MS")) {
-    const long ms = std::strtol(env, nullptr, 10);
-    if (ms > 0) {
-      extra = 1;
-      timeout_ns = static_cast<unsigned long long>(std::min(ms, 1000L)) * 1000000ull;
-    }
+  if (const long ms = switches().test_stall_csr_ms; ms > 0) {
+    extra = 1;
+    timeout_ns = static_cast<unsigned long long>(std::min(ms, 1000L)) * 1000000ull;
   }
   return cudaLaunchKernelEx(&cfg, csr_fused_kernel, idx, R, E, chunk_counts, offsets, perm, inv, status, barrier, mask,
                             k, extra, timeout_ns);

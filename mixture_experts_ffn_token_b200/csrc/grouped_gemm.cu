@@ -890,8 +890,52 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return g_encode;
 }
 
+// The arguments of one encoding: a tensor map is a pure function of them, so
+// an encoded map is reused while they are the same (the same buffers at the
+// same shapes, call after call).
+struct MapKey {
+  const void* base;
+  int rank;
+  cuuint64_t dims[5];
+  cuuint64_t strides[4];
+  cuuint32_t box[5];
+};
+
+bool same_key(const MapKey& a, const MapKey& b) {
+  if (a.base != b.base || a.rank != b.rank) return false;
+  for (int i = 0; i < a.rank; ++i)
+    if (a.dims[i] != b.dims[i] || a.box[i] != b.box[i]) return false;
+  for (int i = 0; i + 1 < a.rank; ++i)
+    if (a.strides[i] != b.strides[i]) return false;
+  return true;
+}
+
+// A small per-thread cache of encoded maps, replaced round-robin.
+constexpr int kMapCacheSize = 32;
+struct MapCache {
+  MapKey key[kMapCacheSize];
+  CUtensorMap map[kMapCacheSize];
+  int used = 0, next = 0;
+};
+thread_local MapCache t_maps;
+
 bool encode_bf16_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
                      const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  MapKey key = {};
+  key.base = base;
+  key.rank = rank;
+  for (int i = 0; i < rank; ++i) {
+    key.dims[i] = dims[i];
+    key.box[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) key.strides[i] = strides_bytes[i];
+  MapCache& c = t_maps;
+  for (int i = 0; i < c.used; ++i) {
+    if (same_key(c.key[i], key)) {
+      *map = c.map[i];
+      return true;
+    }
+  }
   auto enc = encoder();
   if (enc == nullptr) return false;
   const cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
@@ -899,7 +943,17 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, int rank, const cuuint6
                          dims, strides_bytes, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (r != CUDA_SUCCESS) return false;
+  int slot;
+  if (c.used < kMapCacheSize) {
+    slot = c.used++;
+  } else {
+    slot = c.next;
+    c.next = (c.next + 1) % kMapCacheSize;
+  }
+  c.key[slot] = key;
+  c.map[slot] = *map;
+  return true;
 }
 
 template <int PAIR>
@@ -948,22 +1002,11 @@ int max_pair_clusters(size_t smem, int num_sms) {
 // (MOE_B200_FUSED_GATHER=1): the producer warp's lanes copy the tile's rows
 // of x with tile::gather4 instead of a separate gather kernel writing the
 // permuted copy Xp.  Single-CTA tiles only.
-bool fused_gather_requested() {
-  const char* env = std::getenv("MOE_B200_FUSED_GATHER");
-  return env != nullptr && env[0] == '1';
-}
+bool fused_gather_requested() { return switches().fused_gather; }
 
-bool one_box_enabled() {
-  const char* env = std::getenv("MOE_B200_B_ONE_BOX");
-  return !(env != nullptr && env[0] == '0');
-}
+bool one_box_enabled() { return switches().b_one_box; }
 
-int choose_pair(int /*R*/, int /*E*/) {
-  if (const char* env = std::getenv("MOE_B200_CTA_PAIR")) {
-    if (env[0] == '2') return 2;
-  }
-  return 1;
-}
+int choose_pair(int /*R*/, int /*E*/) { return switches().cta_pair; }
 
 template <int MODE, int PAIR, bool GATHER>
 cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const CUtensorMap& mapAh,
@@ -1067,12 +1110,9 @@ cudaError_t prepare(const GroupedGemmArgs& a, CUtensorMap& mapA, CUtensorMap& ma
   // records MOE_DEVICE_ERR_TIMEOUT_GEMM1 | _GEMM2 and ends normally.
   p.extra_arrivals = 0;
   p.dep_timeout_ns = kTimeoutNs;
-  if (const char* env = std::getenv("MOE_B200_TEST_STALL_DOWN_TILES_MS")) {
-    const long ms = std::strtol(env, nullptr, 10);
-    if (ms > 0) {
-      p.extra_arrivals = 1;
-      p.dep_timeout_ns = static_cast<unsigned long long>(std::min(ms, 2000L)) * 1000000ull;
-    }
+  if (const long ms = switches().test_stall_down_ms; ms > 0) {
+    p.extra_arrivals = 1;
+    p.dep_timeout_ns = static_cast<unsigned long long>(std::min(ms, 2000L)) * 1000000ull;
   }
   if (p.b_one_box) {
     // mapB already holds the one-copy view
@@ -1169,10 +1209,8 @@ cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down,
   // where the tensor pipe bounds the launch; MOE_B200_TILE_SCHEDULE=dynamic
   // or =static overrides the choice.
   bool dynamic = up.R < kRidgeRowsPerExpert * up.E;
-  if (const char* env = std::getenv("MOE_B200_TILE_SCHEDULE")) {
-    if (env[0] == 'd') dynamic = true;
-    if (env[0] == 's') dynamic = false;
-  }
+  if (switches().tile_schedule == 'd') dynamic = true;
+  if (switches().tile_schedule == 's') dynamic = false;
   int* sched = dynamic ? arrivals + mega_ffn_counters(up.R, up.E) - 1 : nullptr;
   return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 1, true, GATHER>, mapA, mapB, mapA2, mapB2, mapAh, mapA2h, p,
                             p2,

@@ -7,6 +7,32 @@
 
 namespace moe {
 
+// Runtime switches (environment variables, all optional):
+//   MOE_B200_PDL=0             no programmatic dependent launch
+//   MOE_B200_CSR_FUSED=0       the CSR build as three launches
+//   MOE_B200_SINGLE_LAUNCH=0   the two grouped GEMMs as two launches
+//   MOE_B200_CTA_PAIR=2        CTA-pair GEMM tiles (two launches)
+//   MOE_B200_B_ONE_BOX=0       four copies per B stage tile
+//   MOE_B200_TILE_SCHEDULE=static|dynamic   tile order of the single launch
+//   MOE_B200_FUSED_GATHER=1    the gate_up GEMM gathers its rows of x itself
+//   MOE_B200_TEST_STALL_DOWN_TILES_MS, MOE_B200_TEST_STALL_CSR_MS   test hooks
+//                              that make a bounded wait run out (see the kernels)
+// Every API call takes one snapshot of them (refresh_switches) for all of
+// its launches; switches() returns the calling thread's snapshot.
+struct Switches {
+  bool pdl = true;
+  bool csr_fused = true;
+  long test_stall_csr_ms = 0;
+  bool fused_gather = false;
+  bool b_one_box = true;
+  int cta_pair = 1;
+  long test_stall_down_ms = 0;
+  char tile_schedule = 0;  // 's', 'd', or 0 (chosen by rows per expert)
+  bool single_launch = true;
+};
+void refresh_switches();
+const Switches& switches();
+
 // Launches `kernel` on `stream`, allowing it to overlap the tail of the
 // kernel before it (programmatic dependent launch) unless
 // MOE_B200_PDL=0; every kernel of this library calls griddep_wait() before

@@ -109,10 +109,7 @@ struct WsLayout {
 
 // Whether the two contractions run as one launch (the default) or as two;
 // MOE_B200_SINGLE_LAUNCH=0 selects two launches.
-bool single_launch() {
-  const char* env = std::getenv("MOE_B200_SINGLE_LAUNCH");
-  return !(env != nullptr && env[0] == '0');
-}
+bool single_launch() { return moe::switches().single_launch; }
 
 WsLayout ws_layout(const moe_config_t* c, const Extras* ex = nullptr) {
   const size_t T = static_cast<size_t>(c->num_tokens), H = c->hidden_dim, E = c->num_experts, D = c->moe_dim;
@@ -436,6 +433,7 @@ moe_status_t forward_impl(const moe_config_t* cfg, const moe_extras_t* extras, c
                           const void* gate_up_b, const void* down_w, const void* down_b, void* out, int32_t* idx_out,
                           float* w_out, float* sink_out, void* ws, size_t ws_bytes, cudaStream_t stream,
                           cudaEvent_t const* ev) {
+  moe::refresh_switches();  // one snapshot of the runtime switches for every launch of this call
   const NvtxRange api_range("moe_forward");
   moe_status_t st = validate_config(cfg);
   if (st != MOE_OK) return st;
@@ -549,6 +547,7 @@ const char* moe_status_string(moe_status_t status) {
 }
 
 moe_status_t moe_single_launch_ffn(int32_t* enabled) {
+  moe::refresh_switches();
   if (enabled == nullptr) return MOE_ERR_INVALID_ARGUMENT;
   *enabled = single_launch() ? 1 : 0;
   return MOE_OK;
@@ -565,6 +564,7 @@ moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
 moe_status_t moe_route(const moe_config_t* cfg, const void* logits, const float* expert_bias,
                        const float* global_scale, int32_t* expert_indices, float* expert_weights,
                        float* sink_weights, moe_stream_t stream) {
+  moe::refresh_switches();
   const NvtxRange api_range("moe_route");
   moe_status_t st = validate_config(cfg);
   if (st != MOE_OK) return st;
@@ -582,6 +582,7 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* logits, const float*
 moe_status_t moe_create_indices(const moe_config_t* cfg, const int32_t* expert_indices, int32_t* expert_offsets,
                                 int32_t* permutation, int32_t* inverse, void* workspace, size_t workspace_bytes,
                                 moe_stream_t stream) {
+  moe::refresh_switches();
   const NvtxRange api_range("moe_create_indices");
   moe_status_t st = validate_config(cfg);
   if (st != MOE_OK) return st;
@@ -601,6 +602,7 @@ moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x, const void*
                              const void* down_w, const void* down_b, const int32_t* expert_offsets,
                              const int32_t* permutation, const float* expert_weights, void* out, void* workspace,
                              size_t workspace_bytes, moe_stream_t stream) {
+  moe::refresh_switches();
   const NvtxRange api_range("moe_grouped_ffn");
   moe_status_t st = validate_config(cfg);
   if (st != MOE_OK) return st;
@@ -719,6 +721,7 @@ moe_status_t noalloc_scratch(void** out) {
 extern "C" moe_status_t moe_create_indices_noalloc(const moe_config_t* cfg, const int32_t* expert_indices,
                                                    int32_t* expert_offsets, int32_t* permutation,
                                                    int32_t* inverse, moe_stream_t stream) {
+  moe::refresh_switches();
   moe_status_t st = validate_config(cfg);
   if (st != MOE_OK) return st;
   if (expert_offsets == nullptr) return MOE_ERR_INVALID_ARGUMENT;

@@ -91,3 +91,33 @@ def test_extension_workloads_full_size_every_tile(name):
         if mask is not None:  # some masked tokens too
             sample = np.union1d(sample, np.flatnonzero(mask == 0)[:16])
     run_and_check_ex(wl, seed=0, device_inputs=True, sample_tokens=sample)
+
+
+def test_bound_forward_equals_forward():
+    """abi.BoundForward (arguments marshalled once, the C entry point run on
+    every call) gives moe_forward's and moe_forward_ex's bits, call after call."""
+    wl = SNK.replace(num_tokens=1200)
+    d = to_dev(make_inputs(wl, 9))
+    run = GpuRun(wl, d)
+    out = torch.zeros_like(run.out)
+    ws = torch.empty_like(run.ws)
+    kw = dict(expert_bias=d["expert_bias"], global_scale=d["global_scale"])
+    call = abi.BoundForward(run.cfg, d["x"], d["logits"], d["W_gu"], d["W_d"], out, ws, **kw)
+    for _ in range(2):
+        out.zero_()
+        call()
+        torch.cuda.synchronize()
+        assert torch.equal(out, run.out)
+    wl2 = SNK.replace(num_tokens=1200, num_shared=2, shared_dim=136, mask_frac=0.25)
+    d2 = to_dev(make_inputs(wl2, 10))
+    ex = abi.make_extras(token_mask=d2["token_mask"], shared_gate_up_w=d2["Ws_gu"], shared_down_w=d2["Ws_d"])
+    cfg2 = abi.make_config(wl2)
+    ws2 = torch.empty(abi.moe_workspace_size_ex(cfg2, ex), dtype=torch.uint8, device="cuda")
+    ref = torch.empty((wl2.num_tokens, wl2.hidden_dim), dtype=torch.bfloat16, device="cuda")
+    abi.moe_forward_ex(cfg2, ex, d2["x"], d2["logits"], d2["W_gu"], d2["W_d"], ref, ws2,
+                       expert_bias=d2["expert_bias"], global_scale=d2["global_scale"])
+    got = torch.zeros_like(ref)
+    abi.BoundForward(cfg2, d2["x"], d2["logits"], d2["W_gu"], d2["W_d"], got, ws2, extras=ex,
+                     expert_bias=d2["expert_bias"], global_scale=d2["global_scale"])()
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
