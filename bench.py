@@ -37,6 +37,9 @@ METRIC = "MoE FFN tokens/s and achieved TFLOP/s (or HBM GB/s) vs B200 roofline"
 UNIT = "tokens/s"
 DEFAULT_CONFIG = "mixtral"
 L2_BYTES = 126 * 1024 * 1024
+# e2e: per-step host<->device traffic at or below this runs its copies on the
+# launching stream (latency-bound), above it on double-buffered copy streams
+SMALL_COPY_BYTES = 4 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # the B200 data-sheet figures, for context beside the measured fractions:
 # dense bf16 tensor throughput and HGX HBM3e bandwidth
@@ -418,10 +421,12 @@ def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None, copy_streams=1, 
     from a device token mask) fed from, and returning to, pinned host memory.
     Each step's inputs -- x, the logits and, when there is one, the token
     mask -- sit back to back in one pinned staging buffer and cross to the
-    device in one copy (split by bytes over `copy_streams` streams, so that
-    several copy engines can share it); its output comes back in one copy
-    (split by rows).  Double-buffered, so that step i's copies overlap the
-    compute of its neighbours.  Returns (device time of the whole region in
+    device in one copy; its output comes back in one copy.  Up to
+    SMALL_COPY_BYTES a step the copies run on the launching stream around
+    the call; above it they run on their own streams (split by bytes or rows
+    over `copy_streams` streams, so that several copy engines can share
+    them), double-buffered, so that step i's copies overlap the compute of
+    its neighbours.  Returns (device time of the whole region in
     ms, max over ranks; host->device bytes per step)."""
     T, H = inp["x"].shape
     has_mask = inp["token_mask"] is not None
@@ -455,6 +460,20 @@ def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None, copy_streams=1, 
     d2h = [torch.cuda.Stream() for _ in range(n)]
     bcut = [size * q // n // 256 * 256 for q in range(n)] + [size]  # byte ranges of the split input copy
     cut = [T * q // n for q in range(n + 1)]                         # row ranges of the split output copy
+
+    def region_in_stream(steps):
+        # small transfers: copy in, compute and copy out on the launching
+        # stream, one step after another (no cross-stream events to wait on)
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(steps):
+            b = i % 2
+            stage_d[b].copy_(stage_h, non_blocking=True)
+            calls[b]()
+            out_h[b].copy_(out_d[b], non_blocking=True)
+        stop.record(stream)
+        torch.cuda.synchronize()
+        return start.elapsed_time(stop)
 
     def region(steps):
         in_ready = [[torch.cuda.Event() for _ in range(n)] for _ in range(steps)]
@@ -494,11 +513,17 @@ def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None, copy_streams=1, 
         return start.elapsed_time(stop)
 
     steps = args.steps if steps is None else steps
-    region(max(2, args.warmup))
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    ms = region(steps)
+    # a step whose copies are small (tiny, decode) is bound by host work and
+    # copy latency, not by the link: its copies run on the launching stream;
+    # larger ones overlap their copies with the neighbouring steps' compute
+    in_stream = size + T * H * 2 <= SMALL_COPY_BYTES and copy_streams == 1
+    run = region_in_stream if in_stream else region
+    with torch.cuda.stream(stream):
+        run(max(2, args.warmup))
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ms = run(steps)
     if not torch.equal(out_h[(steps - 1) % 2], out_d[(steps - 1) % 2].cpu()):
         raise RuntimeError("e2e: host copy of the output differs from the device result")
     return max_over_ranks(ms, dist, "cuda"), size
