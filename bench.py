@@ -37,9 +37,9 @@ METRIC = "MoE FFN tokens/s and achieved TFLOP/s (or HBM GB/s) vs B200 roofline"
 UNIT = "tokens/s"
 DEFAULT_CONFIG = "mixtral"
 L2_BYTES = 126 * 1024 * 1024
-# e2e: per-step host<->device traffic at or below this runs its copies on the
-# launching stream (latency-bound), above it on double-buffered copy streams
-SMALL_COPY_BYTES = 4 * 1024 * 1024
+# e2e: a step shorter than this on the device runs its copies on the launching
+# stream (host-bound), a longer one on double-buffered copy streams
+SHORT_STEP_MS = 0.1
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # the B200 data-sheet figures, for context beside the measured fractions:
 # dense bf16 tensor throughput and HGX HBM3e bandwidth
@@ -416,14 +416,16 @@ def timed_steps(step, steps, stream, flush):
     return total
 
 
-def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None, copy_streams=1, steps=None):
+def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None, copy_streams=1, steps=None,
+            device_ms_per_step=None):
     """K steps of moe_forward (moe_forward_ex when `make_ex` builds its extras
     from a device token mask) fed from, and returning to, pinned host memory.
     Each step's inputs -- x, the logits and, when there is one, the token
     mask -- sit back to back in one pinned staging buffer and cross to the
-    device in one copy; its output comes back in one copy.  Up to
-    SMALL_COPY_BYTES a step the copies run on the launching stream around
-    the call; above it they run on their own streams (split by bytes or rows
+    device in one copy; its output comes back in one copy.  For a step
+    shorter than SHORT_STEP_MS on the device (`device_ms_per_step`, from the
+    timed region) the copies run on the launching stream around the call;
+    otherwise they run on their own streams (split by bytes or rows
     over `copy_streams` streams, so that several copy engines can share
     them), double-buffered, so that step i's copies overlap the compute of
     its neighbours.  Returns (device time of the whole region in
@@ -513,10 +515,11 @@ def run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex=None, copy_streams=1, 
         return start.elapsed_time(stop)
 
     steps = args.steps if steps is None else steps
-    # a step whose copies are small (tiny, decode) is bound by host work and
-    # copy latency, not by the link: its copies run on the launching stream;
-    # larger ones overlap their copies with the neighbouring steps' compute
-    in_stream = size + T * H * 2 <= SMALL_COPY_BYTES and copy_streams == 1
+    # a step shorter on the device than SHORT_STEP_MS (tiny) is bound by the
+    # host's work per step, which the cross-stream events of the overlapped
+    # form add to: its copies run on the launching stream; longer steps
+    # overlap their copies with the neighbouring steps' compute
+    in_stream = (device_ms_per_step is not None and device_ms_per_step < SHORT_STEP_MS and copy_streams == 1)
     run = region_in_stream if in_stream else region
     with torch.cuda.stream(stream):
         run(max(2, args.warmup))
@@ -688,7 +691,7 @@ def measure(args, wl, ctx, steps):
     # Copies run on their own streams, double-buffered, so step i's copies
     # overlap the compute of its neighbours.
     e2e_ms, x_h_bytes = run_e2e(args, cfg, inp, kw, ws, stream, dist, make_ex, copy_streams=args.copy_streams,
-                                steps=steps)
+                                steps=steps, device_ms_per_step=ms_per_step)
     e2e_value = job_throughput(world, T, e2e_ms / steps)
     out_bytes = T * H * 2
 
