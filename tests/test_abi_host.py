@@ -162,3 +162,20 @@ def test_extras_validation(lib):
     need = abi.moe_workspace_size(scfg)
     assert lib.moe_forward_ex(by(scfg), by(ex), FAKE, FAKE, None, None, FAKE, None, FAKE, None, FAKE, None, None,
                               None, FAKE, need * 4, None, None) == INVALID
+
+
+def test_switches_are_read_on_every_call(lib, monkeypatch):
+    """Each entry point takes its own snapshot of the MOE_B200_* switches (one
+    pass over the environment), so a change between two calls takes effect
+    at the next call; unrelated and malformed entries are ignored."""
+    monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", "0")
+    assert abi.moe_single_launch_ffn() is False
+    monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", "1")
+    assert abi.moe_single_launch_ffn() is True
+    monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH_X", "0")      # a longer name is another variable
+    monkeypatch.setenv("MOE_B200_", "0")
+    assert abi.moe_single_launch_ffn() is True
+    monkeypatch.delenv("MOE_B200_SINGLE_LAUNCH")
+    assert abi.moe_single_launch_ffn() is True
+    monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", "")        # empty: the default
+    assert abi.moe_single_launch_ffn() is True

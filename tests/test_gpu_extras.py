@@ -34,7 +34,13 @@ def test_token_mask(wl):
 # shared experts' gate_up GEMM reads x directly in each of them.
 GEMM_VARIANTS = {"single_launch": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1"},
                  "two_launches": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "1"},
-                 "cta_pair": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "2"}}
+                 "cta_pair": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "2"},
+                 # row f1 in the routed pass (the shared pass reads x directly,
+                 # and a router weight applied first keeps the gather kernel)
+                 "fused_gather": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1",
+                                  "MOE_B200_FUSED_GATHER": "1"},
+                 "fused_gather_two_launches": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "1",
+                                               "MOE_B200_FUSED_GATHER": "1"}}
 
 
 @pytest.mark.parametrize("variant", sorted(GEMM_VARIANTS))
