@@ -541,17 +541,20 @@ cudaError_t launch_csr_fused(const int32_t* idx, int R, int E, int32_t* chunk_co
     if (err != cudaSuccess) return err;
   }
   // cooperative: the launch fails rather than run CTAs that are not all
-  // resident, which the grid barrier needs
+  // resident, which the grid barrier needs; with programmatic serialization
+  // its CTAs may start while the router drains (they wait in griddep_wait)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(nchunks));
   cfg.blockDim = dim3(kCsrThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() && switches().pdl_coop ? 2 : 1;
   // Test hook for the bounded grid barrier: MOE_B200_TEST_STALL_CSR_MS=<ms>
   // makes every CTA wait for one arrival more than will ever come, giving
   // up after <ms>; the launch then records MOE_DEVICE_ERR_TIMEOUT_CSR and

@@ -1192,17 +1192,22 @@ cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down,
                             static_cast<int>(smem_bytes_for<1>(kMaxExperts)));
   if (err != cudaSuccess) return err;
   // Cooperative: the launch fails rather than run with CTAs that are not
-  // resident, on which a down tile's wait could otherwise depend.
+  // resident, on which a down tile's wait could otherwise depend.  With
+  // programmatic serialization (default) its CTAs may start while the gather
+  // drains: barrier set-up and TMEM allocation overlap it, and every global
+  // read waits in griddep_wait.
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(max_tiles, up.num_sms)));
   cfg.blockDim = dim3(NUM_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() && switches().pdl_coop ? 2 : 1;
   // The last counter is the tile scheduler's (pieces use the ones before it).
   // Dynamic order pays where the weights stream from HBM (rows per expert
   // below the bf16 ridge point of about 256 FLOP/byte), the static order

@@ -9,6 +9,7 @@ namespace moe {
 
 // Runtime switches (environment variables, all optional):
 //   MOE_B200_PDL=0             no programmatic dependent launch
+//   MOE_B200_PDL_COOP=0        none on the two cooperative launches (CSR build, FFN)
 //   MOE_B200_CSR_FUSED=0       the CSR build as three launches
 //   MOE_B200_SINGLE_LAUNCH=0   the two grouped GEMMs as two launches
 //   MOE_B200_CTA_PAIR=2        CTA-pair GEMM tiles (two launches)
@@ -29,6 +30,7 @@ struct Switches {
   long test_stall_down_ms = 0;
   char tile_schedule = 0;  // 's', 'd', or 0 (chosen by rows per expert)
   bool single_launch = true;
+  bool pdl_coop = true;
 };
 void refresh_switches();
 const Switches& switches();
