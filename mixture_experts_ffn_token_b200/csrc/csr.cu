@@ -339,18 +339,17 @@ cudaError_t opt_in_dynamic_smem(const void* func, int bytes) {
   struct Done {
     int dev;
     const void* func;
-    cudaError_t result;
   };
   static std::mutex mu;
-  static std::vector<Done> done;
+  static std::vector<Done> done;  // successful opt-ins only: a failure is retried
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   std::lock_guard<std::mutex> lock(mu);
   for (const Done& d : done)
-    if (d.dev == dev && d.func == func) return d.result;
+    if (d.dev == dev && d.func == func) return cudaSuccess;
   err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  done.push_back({dev, func, err});
+  if (err == cudaSuccess) done.push_back({dev, func});
   return err;
 }
 

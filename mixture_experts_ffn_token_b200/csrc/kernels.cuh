@@ -42,8 +42,8 @@ const Switches& switches();
 bool pdl_enabled();
 
 // Raises the dynamic shared-memory limit of kernel `func` to `bytes` on the
-// current device the first time it is asked for that (device, kernel); later
-// calls return the first call's result without calling the runtime.  Every
+// current device the first time it is asked for that (device, kernel); once
+// that has succeeded, later calls return without calling the runtime.  Every
 // caller passes the kernel's largest possible size, so one opt-in serves all
 // launches.  Thread-safe.
 cudaError_t opt_in_dynamic_smem(const void* func, int bytes);
