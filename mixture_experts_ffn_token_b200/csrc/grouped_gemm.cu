@@ -409,6 +409,19 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoo
   }
 }
 
+// The B tile of one down-GEMM stage: 64 K rows (from kc) x the tile's 256
+// output columns of W_d[e], in one copy or as four 64-column boxes.
+__device__ __forceinline__ void load_down_b(uint32_t sb, const CUtensorMap* map, int one_box, uint32_t bar, int kc,
+                                            const TileCoord& tc) {
+  if (one_box) {
+    tma_load_4d(sb, map, bar, 0, kc, 4 * tc.n, tc.e);
+  } else {
+    const int c0 = tc.n * BN;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * B_BOX_BYTES, map, bar, c0 + 64 * j, kc, tc.e);
+  }
+}
+
 // ------------------------------------------------------------- the kernel
 // FUSED = false: one contraction (MODE) over its tile list.  FUSED = true
 // (single-CTA tiles only): the gate_up contraction (MODE, maps A/B, params p)
@@ -593,14 +606,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // a half tile (at most 64 rows, M = 64 MMAs) copies only 64 rows of A
         const bool half = (PAIR == 1 && tc.rows <= HALF_ROWS) || pair_tail;
         const uint32_t stage_tx = half ? G::STAGE_BYTES - HALF_A_BYTES : G::STAGE_BYTES;
+        // A down tile whose piece is not complete yet issues the B copies of
+        // its first stages (W_d does not depend on h) before it waits, on full
+        // barriers armed with their bytes only (expect_tx, no arrival, so no
+        // stage can complete), and their A copies after the wait.
+        int pre = 0;  // stages of this tile whose B copy went out before the wait
         if constexpr (FUSED) {
           if (ph2) {
             bool got = true;
             if (lane == 0) {
-              got = wait_arrivals(arrivals + tc.piece, arrivals_needed, abort_flag, p.status, p.err_bit,
-                                  p.dep_timeout_ns);
+              if (ld_acquire(arrivals + tc.piece) < arrivals_needed) {
+                for (; pre < nkb && pre < G::STAGES; ++pre) {
+                  const int s = (it + pre) % G::STAGES;
+                  const uint32_t ph = static_cast<uint32_t>((it + pre) / G::STAGES) & 1u;
+                  if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kTimeoutNs)) {
+                    got = false;
+                    break;
+                  }
+                  const uint32_t sb = sbase + s * G::STAGE_BYTES + A_BYTES;
+                  mbar_expect_tx(full0 + 8 * s, 4 * B_BOX_BYTES);
+                  load_down_b(sb, &mapB2, p2.b_one_box, full0 + 8 * s, pre * BK, tc);
+                }
+                if (got)
+                  got = wait_arrivals(arrivals + tc.piece, arrivals_needed, abort_flag, p.status, p.err_bit,
+                                      p.dep_timeout_ns);
+                if (!got) {
+                  // the stages armed so far complete once their B bytes land,
+                  // so the abort drain below can wait for them
+                  for (int j = 0; j < pre; ++j) mbar_arrive(full0 + 8 * ((it + j) % G::STAGES));
+                  it += pre;
+                }
+              }
               if (got) fence_proxy_async_global();  // h stores (generic proxy) before the TMA reads of h
             }
+            pre = bcast(pre);
             if (!bcast(got)) {
               ok = false;
               break;
@@ -629,7 +668,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int s = it % G::STAGES;
           const uint32_t ph = static_cast<uint32_t>(it / G::STAGES) & 1u;
           bool got = true;
-          if (lane == 0) got = mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kTimeoutNs);
+          if (lane == 0 && kb >= pre) got = mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kTimeoutNs);
           if (!bcast(got)) {
             ok = false;
             break;
@@ -663,15 +702,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           } else if (lane == 0) {
             if (FUSED && ph2) {
-              // down tile: h rows of the piece, 256 columns of W_d
-              mbar_arrive_expect_tx(fb, stage_tx);
-              tma_load_2d(sa, half ? &mapA2h : &mapA2, fb, kc, arow);
-              if (p2.b_one_box) {
-                tma_load_4d(sb, &mapB2, fb, 0, kc, 4 * tc.n, tc.e);
+              // down tile: h rows of the piece, 256 columns of W_d (B already
+              // in flight for the first `pre` stages)
+              if (kb < pre) {
+                mbar_arrive_expect_tx(fb, stage_tx - 4 * B_BOX_BYTES);
+                tma_load_2d(sa, half ? &mapA2h : &mapA2, fb, kc, arow);
               } else {
-                const int c0 = tc.n * BN;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * B_BOX_BYTES, &mapB2, fb, c0 + 64 * j, kc, tc.e);
+                mbar_arrive_expect_tx(fb, stage_tx);
+                tma_load_2d(sa, half ? &mapA2h : &mapA2, fb, kc, arow);
+                load_down_b(sb, &mapB2, p2.b_one_box, fb, kc, tc);
               }
             } else if (PAIR == 1 && p.b_one_box) {
               // {64 columns, K, column block, (gate/up,) E} view: one copy lays
