@@ -115,6 +115,7 @@ typedef struct {
 #define MOE_DEVICE_ERR_TIMEOUT_GEMM1  0x4  /* a gate_up GEMM pipeline wait gave up */
 #define MOE_DEVICE_ERR_TIMEOUT_GEMM2  0x8  /* a down GEMM pipeline wait gave up */
 #define MOE_DEVICE_ERR_TIMEOUT_CSR    0x10 /* the one-launch CSR build's grid barrier gave up */
+#define MOE_DEVICE_ERR_LAUNCH         0x20 /* a CTA-pair kernel ran without clusters of two CTAs: nothing computed */
 /* (a wait that gives up inside the single-launch FFN sets both GEMM bits) */
 
 /* Number of events moe_forward_timed() records (one before each stage and

@@ -29,6 +29,7 @@ DEVICE_ERR_CSR = 0x2
 DEVICE_ERR_TIMEOUT_GEMM1 = 0x4
 DEVICE_ERR_TIMEOUT_GEMM2 = 0x8
 DEVICE_ERR_TIMEOUT_CSR = 0x10
+DEVICE_ERR_LAUNCH = 0x20
 NUM_STAGE_EVENTS = 9
 STAGE_NAMES = ("router", "csr_count", "csr_scan", "csr_scatter", "gather", "gemm_gate_up", "gemm_down", "combine")
 

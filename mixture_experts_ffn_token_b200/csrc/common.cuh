@@ -246,6 +246,12 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   return r;
 }
 
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t n;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+  return n;
+}
+
 // All threads of both CTAs of the cluster; release/acquire orders the shared
 // memory each CTA wrote before it against the other's reads after it.
 __device__ __forceinline__ void cluster_sync() {

@@ -40,7 +40,8 @@
 // (per-piece arrival counters, release/acquire).  CTAs take tiles with a
 // static stride or, below 256 rows per expert, from an atomic counter.  A
 // variant on CTA pairs (tcgen05 cta_group::2, 256x256 tiles, M = 128 over
-// the pair for pieces of at most 128 rows, two launches) is kept selectable.
+// the pair for pieces of at most 128 rows; in the single launch with the
+// static tile order, or as two launches) is kept selectable.
 //
 // Weights are read in their stored [K, N] (N-contiguous) layout: the B
 // operand is MN-major, which tcgen05 supports for 16-bit types, so no
@@ -53,6 +54,7 @@
 #include <algorithm>
 #include <cstdlib>
 #include <mutex>
+#include <vector>
 
 #include "kernels.cuh"
 
@@ -436,7 +438,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         const __grid_constant__ CUtensorMap mapA2, const __grid_constant__ CUtensorMap mapB2,
                         const __grid_constant__ CUtensorMap mapAh, const __grid_constant__ CUtensorMap mapA2h,
                         const GemmParams p, const GemmParams p2, int* arrivals, int* sched) {
-  static_assert(!FUSED || (PAIR == 1 && MODE != MODE_DOWN), "the fused form is gate_up then down, one CTA a tile");
+  static_assert(!FUSED || MODE != MODE_DOWN, "the fused form is gate_up then down");
   static_assert(!GATHER || (PAIR == 1 && MODE != MODE_DOWN), "rows are gathered for gate_up tiles of one CTA");
   using G = Geo<PAIR>;
   extern __shared__ uint8_t smem_raw[];
@@ -450,7 +452,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t drain_bar = tempty0 + 16;            // 1 mbarrier
   const uint32_t ring_full0 = drain_bar + 8;          // kTileRing mbarriers (FUSED)
   const uint32_t ring_empty0 = ring_full0 + 8 * kTileRing;  // kTileRing mbarriers (FUSED)
-  static_assert((2 * G::STAGES + 5 + (FUSED ? 2 * kTileRing : 0)) * 8 <= 256,
+  // the dynamic tile order (and its ring of tile numbers) is for one CTA a tile
+  constexpr bool kRing = FUSED && PAIR == 1;
+  static_assert((2 * G::STAGES + 5 + (kRing ? 2 * kTileRing : 0)) * 8 <= 256,
                 "mbarriers overflow their part of the control block");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 256);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 260);
@@ -464,6 +468,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if constexpr (PAIR == 2) {
+    // the pair's tcgen05 operations need a cluster of exactly two CTAs
+    if (cluster_nctarank() != 2) {
+      if (threadIdx.x == 0) atomicOr(p.status, MOE_DEVICE_ERR_LAUNCH);
+      return;
+    }
+  }
   const uint32_t rank = PAIR == 2 ? cluster_ctarank() : 0u;  // 0 = leader of the pair
   const bool leader = rank == 0;
 
@@ -477,7 +488,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(tempty0 + 8 * a, 32 * NUM_EPI_WARPS * PAIR);
     }
     mbar_init(drain_bar, 1);
-    if constexpr (FUSED) {
+    if constexpr (kRing) {
       for (int i = 0; i < kTileRing; ++i) {
         mbar_init(ring_full0 + 8 * i, 1);
         mbar_init(ring_empty0 + 8 * i, 1 + NUM_EPI_WARPS);  // the MMA thread and one lane per epilogue warp
@@ -548,8 +559,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int tile_stride = gridDim.x / PAIR;
   // down tiles of a piece wait for this many arrivals (one per epilogue warp
   // of each of the piece's gate_up tiles)
-  const int arrivals_needed = NUM_EPI_WARPS * p.n_tiles + p.extra_arrivals;
-  const bool dyn = FUSED && sched != nullptr;  // dynamic tile order
+  const int arrivals_needed = NUM_EPI_WARPS * PAIR * p.n_tiles + p.extra_arrivals;
+  const bool dyn = kRing && sched != nullptr;  // dynamic tile order
 
   if (warp == 0) {
     if (GATHER || lane == 0) {
@@ -616,7 +627,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             bool got = true;
             if (lane == 0) {
               if (ld_acquire(arrivals + tc.piece) < arrivals_needed) {
-                for (; pre < nkb && pre < G::STAGES; ++pre) {
+                // (one CTA a tile only: a pair's leader counts both CTAs' bytes)
+                for (; PAIR == 1 && pre < nkb && pre < G::STAGES; ++pre) {
                   const int s = (it + pre) % G::STAGES;
                   const uint32_t ph = static_cast<uint32_t>((it + pre) / G::STAGES) & 1u;
                   if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kTimeoutNs)) {
@@ -701,7 +713,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
             }
           } else if (lane == 0) {
-            if (FUSED && ph2) {
+            if (FUSED && ph2 && PAIR == 2) {
+              // down tile of a CTA pair: each CTA copies its rows of h (128,
+              // or 64 in a pair tail) and its half of the tile's 256 columns
+              // of W_d; the leader expects both CTAs' bytes
+              if (leader) mbar_arrive_expect_tx(full0 + 8 * s, 2 * stage_tx);
+              tma_load_2d_pair(sa, half ? &mapA2h : &mapA2, fb, kc, arow);
+              if (p2.b_one_box) {
+                tma_load_4d_pair(sb, &mapB2, fb, 0, kc, 4 * tc.n + 2 * static_cast<int>(rank), tc.e);
+              } else {
+                const int c0 = tc.n * BN + static_cast<int>(rank) * 128;
+                tma_load_3d_pair(sb, &mapB2, fb, c0, kc, tc.e);
+                tma_load_3d_pair(sb + B_BOX_BYTES, &mapB2, fb, c0 + 64, kc, tc.e);
+              }
+            } else if (FUSED && ph2) {
               // down tile: h rows of the piece, 256 columns of W_d (B already
               // in flight for the first `pre` stages)
               if (kb < pre) {
@@ -1001,17 +1026,21 @@ constexpr size_t smem_bytes_for(int E) {
          2 * static_cast<size_t>(E + 1) * 4 + 16 + NUM_EPI_WARPS * kStageWarpBytes;
 }
 
-// Clusters of two that can be resident at once, looked up once per device
-// (occupancy depends on the device) and kernel.
-template <int MODE>
-int max_pair_clusters(size_t smem, int num_sms) {
-  constexpr int kDevices = 64;
+// Clusters of two of kernel `func` that can be resident at once, looked up
+// once per device (occupancy depends on the device) and kernel.
+int max_pair_clusters(const void* func, size_t smem, int num_sms) {
+  struct Entry {
+    int dev;
+    const void* func;
+    int n;
+  };
   static std::mutex mu;
-  static int cached[kDevices] = {};
+  static std::vector<Entry> cache;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) return num_sms / 2;
+  if (cudaGetDevice(&dev) != cudaSuccess) return num_sms / 2;
   std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev] > 0) return cached[dev];
+  for (const Entry& c : cache)
+    if (c.dev == dev && c.func == func) return c.n;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1024,9 +1053,8 @@ int max_pair_clusters(size_t smem, int num_sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<MODE, 2, false, false>, &cfg) != cudaSuccess || n <= 0)
-    n = num_sms / 2;
-  cached[dev] = n;
+  if (cudaOccupancyMaxActiveClusters(&n, func, &cfg) != cudaSuccess || n <= 0) return num_sms / 2;
+  cache.push_back({dev, func, n});
   return n;
 }
 
@@ -1062,8 +1090,9 @@ cudaError_t launch_with(const CUtensorMap& mapA, const CUtensorMap& mapB, const 
                                                                                       mapAh, p, p, nullptr, nullptr);
     return cudaGetLastError();
   } else {
-    const int clusters =
-        static_cast<int>(std::min<int64_t>(max_tiles, max_pair_clusters<MODE>(smem_bytes_for<2>(kMaxExperts), num_sms)));
+    const int clusters = static_cast<int>(std::min<int64_t>(
+        max_tiles, max_pair_clusters(reinterpret_cast<const void*>(grouped_gemm_kernel<MODE, 2, false, false>),
+                                     smem_bytes_for<2>(kMaxExperts), num_sms)));
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1261,6 +1290,57 @@ cudaError_t launch_fused(const GroupedGemmArgs& up, const GroupedGemmArgs& down,
                             arrivals, sched);
 }
 
+// Both contractions in one launch on CTA pairs (tcgen05 cta_group::2):
+// 256-row pieces, each CTA of a pair copying its rows of A and its half of
+// B, static tile order.  Cooperative and clustered: the launch fails rather
+// than run with clusters that are not all resident.
+template <int MODE>
+cudaError_t launch_fused_pair(const GroupedGemmArgs& up, const GroupedGemmArgs& down, int* arrivals,
+                              cudaStream_t stream) {
+  if (up.R == 0) return cudaSuccess;
+  CUtensorMap mapA, mapAh, mapB, mapA2, mapA2h, mapB2;
+  GemmParams p, p2;
+  cudaError_t err = prepare<MODE>(up, mapA, mapAh, mapB, p, true);
+  if (err != cudaSuccess) return err;
+  err = prepare<MODE_DOWN>(down, mapA2, mapA2h, mapB2, p2, true);
+  if (err != cudaSuccess) return err;
+  p.err_bit = p2.err_bit = MOE_DEVICE_ERR_TIMEOUT_GEMM1 | MOE_DEVICE_ERR_TIMEOUT_GEMM2;
+  const int64_t max_pieces = p.R / Geo<2>::PIECE + std::min(p.E, p.R);
+  const int64_t max_tiles = max_pieces * (p.n_tiles + p2.n_tiles);
+  const size_t smem = smem_bytes_for<2>(p.E);
+  const void* kernel = reinterpret_cast<const void*>(grouped_gemm_kernel<MODE, 2, true, false>);
+  err = opt_in_dynamic_smem(kernel, static_cast<int>(smem_bytes_for<2>(kMaxExperts)));
+  if (err != cudaSuccess) return err;
+  const int clusters = static_cast<int>(
+      std::min<int64_t>(max_tiles, max_pair_clusters(kernel, smem_bytes_for<2>(kMaxExperts), up.num_sms)));
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[3];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeClusterDimension;
+  attr[n].val.clusterDim.x = 2;
+  attr[n].val.clusterDim.y = 1;
+  attr[n].val.clusterDim.z = 1;
+  ++n;
+  if (switches().pair_coop) {
+    attr[n].id = cudaLaunchAttributeCooperative;
+    attr[n].val.cooperative = 1;
+    ++n;
+  }
+  if (pdl_enabled() && switches().pdl_coop) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, 2, true, false>, mapA, mapB, mapA2, mapB2, mapAh,
+                            mapA2h, p, p2, arrivals, static_cast<int*>(nullptr));
+}
+
 }  // namespace
 
 bool tensor_map_encoder_available() { return encoder() != nullptr; }
@@ -1283,6 +1363,9 @@ cudaError_t launch_mega_ffn(const GroupedGemmArgs& up, const GroupedGemmArgs& do
   if (up.gather)
     return up.gate_up_format == 0 ? launch_fused<MODE_GATE_UP_CONCAT, true>(up, down, arrivals, stream)
                                   : launch_fused<MODE_GATE_UP_INTERLEAVED, true>(up, down, arrivals, stream);
+  if (choose_pair(up.R, up.E) == 2)
+    return up.gate_up_format == 0 ? launch_fused_pair<MODE_GATE_UP_CONCAT>(up, down, arrivals, stream)
+                                  : launch_fused_pair<MODE_GATE_UP_INTERLEAVED>(up, down, arrivals, stream);
   return up.gate_up_format == 0 ? launch_fused<MODE_GATE_UP_CONCAT, false>(up, down, arrivals, stream)
                                 : launch_fused<MODE_GATE_UP_INTERLEAVED, false>(up, down, arrivals, stream);
 }

@@ -31,6 +31,7 @@ struct Switches {
   char tile_schedule = 0;  // 's', 'd', or 0 (chosen by rows per expert)
   bool single_launch = true;
   bool pdl_coop = true;
+  bool pair_coop = true;
 };
 void refresh_switches();
 const Switches& switches();

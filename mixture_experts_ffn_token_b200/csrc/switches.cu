@@ -41,6 +41,7 @@ void refresh_switches() {
     else if (is("TILE_SCHEDULE")) s.tile_schedule = (v[0] == 'd' || v[0] == 's') ? v[0] : 0;
     else if (is("SINGLE_LAUNCH")) s.single_launch = v[0] != '0';
     else if (is("PDL_COOP")) s.pdl_coop = v[0] != '0';
+    else if (is("PAIR_COOP")) s.pair_coop = v[0] != '0';
   }
   t_switches = s;
   t_switches_read = true;

@@ -49,6 +49,10 @@ VARIANTS = {"single_launch": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR"
                                        "MOE_B200_B_ONE_BOX": "0"},
             "two_launches": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "1", "MOE_B200_B_ONE_BOX": "1"},
             "two_launches_cta_pair": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "2"},
+            "single_launch_cta_pair": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "2",
+                                       "MOE_B200_B_ONE_BOX": "1"},
+            "single_launch_cta_pair_four_box": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "2",
+                                                "MOE_B200_B_ONE_BOX": "0"},
             # row f1: the gate_up GEMM gathers its rows of x itself (tile::gather4)
             "single_launch_fused_gather": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1",
                                            "MOE_B200_B_ONE_BOX": "1", "MOE_B200_FUSED_GATHER": "1"},
@@ -421,11 +425,13 @@ def test_forward_full_size_every_tile(name, monkeypatch):
         check_full_size_run(wl, inp, route_ref, tokens, ref)
 
 
+@pytest.mark.parametrize("variant", ["two_launches_cta_pair", "single_launch_cta_pair"])
 @pytest.mark.parametrize("name", ["mixtral", "sink"])
-def test_forward_full_size_every_tile_cta_pair(name, monkeypatch):
-    """The selectable CTA-pair variant at full size: 256-row pieces and
-    M = 128 pair tails over every expert of the workload."""
-    set_variant(monkeypatch, "two_launches_cta_pair")
+def test_forward_full_size_every_tile_cta_pair(name, variant, monkeypatch):
+    """The selectable CTA-pair variants at full size, as two launches and as
+    one: 256-row pieces and M = 128 pair tails over every expert of the
+    workload."""
+    set_variant(monkeypatch, variant)
     wl = WORKLOADS[name]
     inp, route_ref, tokens, ref = full_size_reference(wl)
     check_full_size_run(wl, inp, route_ref, tokens, ref)

@@ -18,12 +18,13 @@ GPT = WORKLOADS["gptoss"].replace(num_tokens=96, hidden_dim=328, num_experts=16,
 TIMEOUT_BITS = abi.DEVICE_ERR_TIMEOUT_GEMM1 | abi.DEVICE_ERR_TIMEOUT_GEMM2
 
 
-@pytest.mark.parametrize("order", ["static", "dynamic"])
+@pytest.mark.parametrize("order", ["static", "dynamic", "static_cta_pair"])
 @pytest.mark.parametrize("wl", [SINK, GPT], ids=["sink", "gptoss"])
 def test_down_tile_wait_gives_up_and_recovers(wl, order, monkeypatch):
     d = to_dev(make_inputs(wl, 21))
     monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", "1")
-    monkeypatch.setenv("MOE_B200_TILE_SCHEDULE", order)
+    monkeypatch.setenv("MOE_B200_TILE_SCHEDULE", order.split("_")[0])
+    monkeypatch.setenv("MOE_B200_CTA_PAIR", "2" if order.endswith("cta_pair") else "1")
     monkeypatch.setenv("MOE_B200_TEST_STALL_DOWN_TILES_MS", "20")
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
