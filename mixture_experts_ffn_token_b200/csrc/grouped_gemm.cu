@@ -37,11 +37,15 @@
 // By default both contractions run in ONE cooperative launch (FUSED): the
 // tile list is every gate_up tile, then every down tile; a down tile of a
 // piece starts once all gate_up tiles of that piece have published their h
-// (per-piece arrival counters, release/acquire).  CTAs take tiles with a
-// static stride or, below 256 rows per expert, from an atomic counter.  A
+// (per-piece arrival counters, release/acquire); while it waits, its
+// producer already copies the B stages the ring can hold (W_d does not
+// depend on h).  CTAs take tiles with a static stride or, below 256 rows
+// per expert, from an atomic counter.  A
 // variant on CTA pairs (tcgen05 cta_group::2, 256x256 tiles, M = 128 over
 // the pair for pieces of at most 128 rows; in the single launch with the
-// static tile order, or as two launches) is kept selectable.
+// static tile order, or as two launches) is kept selectable, and so is the
+// gate_up GEMM gathering its rows of x itself (GATHER: tile::gather4 from
+// every lane of the producer warp) instead of reading the gathered copy.
 //
 // Weights are read in their stored [K, N] (N-contiguous) layout: the B
 // operand is MN-major, which tcgen05 supports for 16-bit types, so no
