@@ -721,9 +721,18 @@ def measure(args, wl, ctx, steps):
         # the "gate_up" stage is the single launch of both GEMMs; "down" is empty
         names = [{"gemm_gate_up": "mega_ffn", "gemm_down": "(fused)", "shared_gemm_gate_up": "shared_mega_ffn",
                   "shared_gemm_down": "(shared fused)"}.get(n, n) for n in names]
+    csr_fused = csr_fused_active(wl, torch.cuda.get_device_properties(local).multi_processor_count)
+    small = wl.num_tokens * wl.top_k <= 2048 and wl.num_experts <= 512
+    if small:
+        # routing and the CSR build are one kernel, timed as the router stage
+        names = [{"router": "route_csr_small", "csr_count": "(csr in route)", "csr_scan": "(csr scan in route)",
+                  "csr_scatter": "(csr scatter in route)"}.get(n, n) for n in names]
+    elif csr_fused:
+        # the one-launch CSR build is timed as the first CSR stage
+        names = [{"csr_count": "csr_build", "csr_scan": "(csr scan in build)",
+                  "csr_scatter": "(csr scatter in build)"}.get(n, n) for n in names]
     flops = wl.flops()
     wbytes, used = touched_expert_bytes(wl, idx)
-    csr_fused = csr_fused_active(wl, torch.cuda.get_device_properties(local).multi_processor_count)
     fused_gather = os.environ.get("MOE_B200_FUSED_GATHER", "0").startswith("1")
     dom_name = names[dom]
     clock_summary = clocks.summary()

@@ -35,6 +35,7 @@ def test_token_mask(wl):
 GEMM_VARIANTS = {"single_launch": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1"},
                  "two_launches": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "1"},
                  "cta_pair": {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "2"},
+                 "single_launch_cta_pair": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "2"},
                  # row f1 in the routed pass (the shared pass reads x directly,
                  # and a router weight applied first keeps the gather kernel)
                  "fused_gather": {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "1",

@@ -273,11 +273,14 @@ def test_sink_router_extremes():
 
 @pytest.mark.parametrize("fused", ["1", "0"])
 @pytest.mark.parametrize("T,E,k", [(1, 1, 1), (1000, 16, 4), (4096, 128, 6), (7, 1024, 3), (50000, 8, 2),
-                                   (8192, 1024, 6), (160000, 64, 2)])
+                                   (8192, 1024, 6), (160000, 64, 2),
+                                   # 148 and 149 chunks of 2048 slots: the most the
+                                   # one-launch form takes on a 148-SM B200, and one more
+                                   (151552, 16, 2), (151553, 16, 2)])
 def test_create_indices(T, E, k, fused, monkeypatch):
     """Both forms of the CSR build (one cooperative launch, or count -> scan
-    -> scatter) against the oracle's counting sort, bit for bit.  160000 x 2
-    slots are more chunks than SMs, so that case always takes three launches."""
+    -> scatter) against the oracle's counting sort, bit for bit.  Problems of
+    more chunks than SMs always take three launches."""
     monkeypatch.setenv("MOE_B200_CSR_FUSED", fused)
     g = torch.Generator().manual_seed(T + E)
     idx = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32) if T < 5000 else \
