@@ -767,6 +767,12 @@ def measure(args, wl, ctx, steps):
 PER_CONFIG = ("tiny", "gptoss", "sink", "decode")
 
 
+def per_config_enabled(flag, world):
+    """--per-config / --no-per-config, else on with one GPU only (with
+    several GPUs every rank would hold its GPU through four more workloads)."""
+    return flag if flag is not None else world == 1
+
+
 def compact(line):
     """The per-config entry: the figures of a full line that describe one workload."""
     keep = ("value", "unit", "ms_per_step", "steps", "tflops", "weight_gbs", "experts_touched", "roofline", "e2e",
@@ -793,8 +799,7 @@ def run_gpu(args, wl):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, inp)
     del inp
-    per_config = args.per_config if args.per_config is not None else world == 1
-    if per_config:
+    if per_config_enabled(args.per_config, world):
         line["per_config"] = {}
         for name in PER_CONFIG:
             if name == wl.name:

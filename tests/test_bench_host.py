@@ -134,3 +134,11 @@ def test_launches_per_step():
     # shared experts reading x directly: index kernel + single launch
     assert bench.launches_per_step(W["sink_shared"], True, csr_fused=True) == 7
     assert bench.csr_fused_active(W["sink"], 148) and not bench.csr_fused_active(W["sink"], 16)
+
+
+def test_per_config_default():
+    assert bench.per_config_enabled(None, 1) is True
+    assert bench.per_config_enabled(None, 8) is False
+    assert bench.per_config_enabled(True, 4) is True
+    assert bench.per_config_enabled(False, 1) is False
+    assert set(bench.PER_CONFIG) == {"tiny", "gptoss", "sink", "decode"}
