@@ -63,7 +63,7 @@ def oracle_ffn(wl, inp, idx, w, tokens=None):
                              wl.alpha, wl.limit, tokens=tokens)
 
 
-class GpuRun:
+class LayerRun:
     """One moe_forward call with every output kept for comparison."""
 
     def __init__(self, wl, d, out_guard=0):
@@ -99,7 +99,7 @@ def run_and_check(wl, seed=0, device_inputs=False, sample_tokens=None, out_guard
     """moe_forward against the oracle: routing bit-exact, weights 1e-5, output FFN_TOL."""
     inp = make_inputs(wl, seed, device="cuda" if device_inputs else "cpu")
     d = to_dev(inp)
-    run = GpuRun(wl, d, out_guard=out_guard)
+    run = LayerRun(wl, d, out_guard=out_guard)
     assert run.status == 0, f"device status {run.status:#x}"
     idx_ref, w_ref, s_ref = oracle_route(wl, inp)
     idx = run.idx.cpu().numpy()

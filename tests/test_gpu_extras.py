@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import GpuRun, every_tile_tokens, oracle_route, run_and_check_ex, to_dev
+from gpu_helpers import LayerRun, every_tile_tokens, oracle_route, run_and_check_ex, to_dev
 from mixture_experts_ffn_token_b200 import abi
 from mixture_experts_ffn_token_b200.workloads import WORKLOADS, make_inputs
 
@@ -70,7 +70,7 @@ def test_no_extras_equals_forward():
     """moe_forward_ex with no extensions gives moe_forward's output bit for bit."""
     wl = SNK.replace(num_tokens=1200)
     d = to_dev(make_inputs(wl, 6))
-    run = GpuRun(wl, d)
+    run = LayerRun(wl, d)
     out = torch.empty_like(run.out)
     sink = torch.empty_like(run.sink)
     events = [torch.cuda.Event(enable_timing=True) for _ in range(abi.NUM_STAGE_EVENTS_EX)]
@@ -105,7 +105,7 @@ def test_bound_forward_equals_forward():
     every call) gives moe_forward's and moe_forward_ex's bits, call after call."""
     wl = SNK.replace(num_tokens=1200)
     d = to_dev(make_inputs(wl, 9))
-    run = GpuRun(wl, d)
+    run = LayerRun(wl, d)
     out = torch.zeros_like(run.out)
     ws = torch.empty_like(run.ws)
     kw = dict(expert_bias=d["expert_bias"], global_scale=d["global_scale"])

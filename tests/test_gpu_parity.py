@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import (FFN_TOL, GpuRun, check_weights, every_tile_tokens, ffn_error, oracle_ffn, oracle_route,
+from gpu_helpers import (FFN_TOL, LayerRun, check_weights, every_tile_tokens, ffn_error, oracle_ffn, oracle_route,
                          run_and_check, to_dev)
 from mixture_experts_ffn_token_b200 import abi
 from mixture_experts_ffn_token_b200.workloads import WORKLOADS, make_inputs
@@ -106,7 +106,7 @@ def test_single_launch_equals_two_launches(name, monkeypatch):
         monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", single)
         monkeypatch.setenv("MOE_B200_B_ONE_BOX", one_box)
         monkeypatch.setenv("MOE_B200_TILE_SCHEDULE", order)
-        run = GpuRun(wl, d)
+        run = LayerRun(wl, d)
         assert run.status == 0
         outs.append(run.out.clone())
     for o in outs[1:]:
@@ -124,7 +124,7 @@ def test_cta_pair_one_copy_equals_two_copies(name, monkeypatch):
     outs = []
     for one_box in ("1", "0"):
         monkeypatch.setenv("MOE_B200_B_ONE_BOX", one_box)
-        run = GpuRun(wl, d)
+        run = LayerRun(wl, d)
         assert run.status == 0
         outs.append(run.out.clone())
     assert torch.equal(outs[0], outs[1])
@@ -139,7 +139,7 @@ def test_programmatic_launch_changes_nothing(name, monkeypatch):
     outs = []
     for pdl in ("1", "0"):
         monkeypatch.setenv("MOE_B200_PDL", pdl)
-        run = GpuRun(wl, d)
+        run = LayerRun(wl, d)
         assert run.status == 0
         outs.append((run.out.clone(), run.idx.clone(), run.w.clone()))
     for a, b in zip(outs[0], outs[1]):
@@ -197,7 +197,7 @@ def test_all_tokens_on_one_expert():
     inp = make_inputs(wl, 4)
     inp["logits"][:, 5] += 100.0        # expert 5 first for every token; every other segment is short or empty
     d = to_dev(inp)
-    run = GpuRun(wl, d)
+    run = LayerRun(wl, d)
     idx_ref, w_ref, _ = oracle_route(wl, inp)
     assert (idx_ref[:, 0] == 5).all()
     assert np.array_equal(run.idx.cpu().numpy(), idx_ref)
@@ -320,7 +320,7 @@ def test_stages_compose_to_forward():
     wl = SMALL["gptoss_small"]
     inp = make_inputs(wl, 6)
     d = to_dev(inp)
-    run = GpuRun(wl, d)
+    run = LayerRun(wl, d)
     T, k, E = wl.num_tokens, wl.top_k, wl.num_experts
     cfg = run.cfg
     ws = torch.empty_like(run.ws)
@@ -335,14 +335,14 @@ def test_stages_compose_to_forward():
     torch.cuda.synchronize()
     assert torch.equal(idx, run.idx) and torch.equal(w, run.w)
     assert torch.equal(out, run.out)
-    again = GpuRun(wl, d)
+    again = LayerRun(wl, d)
     assert torch.equal(again.out, run.out)         # deterministic
 
 
 def test_forward_timed_matches_forward():
     wl = SMALL["sink_small"]
     d = to_dev(make_inputs(wl, 8))
-    run = GpuRun(wl, d)
+    run = LayerRun(wl, d)
     events = [torch.cuda.Event(enable_timing=True) for _ in range(abi.NUM_STAGE_EVENTS)]
     out = torch.empty_like(run.out)
     sink = torch.empty_like(run.sink)
@@ -400,7 +400,7 @@ def full_size_reference(wl):
 
 def check_full_size_run(wl, inp, route_ref, tokens, ref):
     idx_ref, w_ref, s_ref = route_ref
-    run = GpuRun(wl, inp, out_guard=64)
+    run = LayerRun(wl, inp, out_guard=64)
     assert run.status == 0, f"device status {run.status:#x}"
     assert np.array_equal(run.idx.cpu().numpy(), idx_ref)
     check_weights(run.w.cpu().numpy(), w_ref)
@@ -449,10 +449,10 @@ def test_full_size_runs_are_bit_identical(name, order, monkeypatch):
     monkeypatch.setenv("MOE_B200_TILE_SCHEDULE", order)
     wl = WORKLOADS[name]
     d = to_dev(make_inputs(wl, 21, device="cuda"))
-    first = GpuRun(wl, d)
+    first = LayerRun(wl, d)
     assert first.status == 0
     for _ in range(2):
-        again = GpuRun(wl, d)
+        again = LayerRun(wl, d)
         assert again.status == 0
         assert torch.equal(first.out, again.out) and torch.equal(first.idx, again.idx)
         assert torch.equal(first.w, again.w)
@@ -483,7 +483,7 @@ def test_cuda_graph_capture(name):
     dependent launches included); every replay gives the eager result."""
     wl = SMALL[name]
     d = to_dev(make_inputs(wl, 16))
-    eager = GpuRun(wl, d)
+    eager = LayerRun(wl, d)
     assert eager.status == 0
     T, H, k, S = wl.num_tokens, wl.hidden_dim, wl.top_k, wl.num_sink
     ws = torch.empty_like(eager.ws)
@@ -511,7 +511,7 @@ def test_stage_events_inside_a_cuda_graph():
     pair, and the stage time is positive and shorter than the whole step."""
     wl = SMALL["sink_small"]
     d = to_dev(make_inputs(wl, 17))
-    eager = GpuRun(wl, d)
+    eager = LayerRun(wl, d)
     ws = torch.empty_like(eager.ws)
     out = torch.empty_like(eager.out)
     kw = dict(expert_bias=d["expert_bias"], global_scale=d["global_scale"])
@@ -581,9 +581,9 @@ def test_fused_gather_equals_gather_kernel(name, order, monkeypatch):
     for single in ("1", "0"):
         monkeypatch.setenv("MOE_B200_SINGLE_LAUNCH", single)
         monkeypatch.setenv("MOE_B200_FUSED_GATHER", "0")
-        ref = GpuRun(wl, d)
+        ref = LayerRun(wl, d)
         monkeypatch.setenv("MOE_B200_FUSED_GATHER", "1")
-        got = GpuRun(wl, d)
+        got = LayerRun(wl, d)
         assert ref.status == 0 and got.status == 0
         assert torch.equal(got.out, ref.out), (name, single)
 
@@ -595,9 +595,9 @@ def test_fused_gather_full_size_equals_gather_kernel(name, monkeypatch):
     wl = WORKLOADS[name]
     d = to_dev(make_inputs(wl, 0, device="cuda"))
     monkeypatch.setenv("MOE_B200_FUSED_GATHER", "0")
-    ref = GpuRun(wl, d)
+    ref = LayerRun(wl, d)
     monkeypatch.setenv("MOE_B200_FUSED_GATHER", "1")
-    got = GpuRun(wl, d)
+    got = LayerRun(wl, d)
     assert ref.status == 0 and got.status == 0
     assert torch.equal(got.out, ref.out)
 
@@ -609,8 +609,8 @@ def test_csr_forms_give_the_same_forward(name, monkeypatch):
     wl = WORKLOADS[name]
     d = to_dev(make_inputs(wl, 3, device="cuda"))
     monkeypatch.setenv("MOE_B200_CSR_FUSED", "1")
-    a = GpuRun(wl, d)
+    a = LayerRun(wl, d)
     monkeypatch.setenv("MOE_B200_CSR_FUSED", "0")
-    b = GpuRun(wl, d)
+    b = LayerRun(wl, d)
     assert a.status == 0 and b.status == 0
     assert torch.equal(a.out, b.out) and torch.equal(a.idx, b.idx)

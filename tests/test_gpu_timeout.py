@@ -7,7 +7,7 @@ than any gate_up tile will deliver (nothing faults, traps or hangs)."""
 import pytest
 import torch
 
-from gpu_helpers import GpuRun, run_and_check, to_dev
+from gpu_helpers import LayerRun, run_and_check, to_dev
 from mixture_experts_ffn_token_b200 import abi
 from mixture_experts_ffn_token_b200.workloads import WORKLOADS, make_inputs
 
@@ -28,7 +28,7 @@ def test_down_tile_wait_gives_up_and_recovers(wl, order, monkeypatch):
     monkeypatch.setenv("MOE_B200_TEST_STALL_DOWN_TILES_MS", "20")
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
-    run = GpuRun(wl, d)
+    run = LayerRun(wl, d)
     stop.record()
     torch.cuda.synchronize()
     assert run.status & TIMEOUT_BITS == TIMEOUT_BITS, f"status {run.status:#x}"
