@@ -264,6 +264,14 @@ def kernel_traffic(workload, kernel):
     return ent.get("bytes_per_launch")
 
 
+def dram_frac(traffic, kernel_ms, peaks):
+    """The dominant kernel's measured DRAM traffic per launch over its live
+    time, as a fraction of the measured HBM copy bandwidth. Beside a
+    tensor-bound `frac` it shows how close the kernel also runs to the
+    memory roof (a kernel near the ridge point needs both at once)."""
+    return traffic / (kernel_ms / 1e3) / (peaks["hbm_gbs"] * 1e9)
+
+
 _C_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'|//[^\n]*|/\*.*?\*/|\s+', re.S)
 
 
@@ -739,6 +747,8 @@ def measure(args, wl, ctx, steps):
     roof = roofline(wl, dom_name, kernel_ms, peaks, peak_kind, clock_summary, used, region_s=region_ms / 1e3)
     roof["kernel"] = dom_name
     roof["traffic"] = kernel_traffic(wl.name, dom_name)
+    if roof["traffic"] is not None:
+        roof["dram_frac"] = dram_frac(roof["traffic"], kernel_ms, peaks)
     roof["kernel_ms"] = kernel_ms                # live, in the timed region
     roof["kernel_ms_stage_region"] = stage_ms[dom]
 

@@ -117,6 +117,12 @@ def test_roofline_arithmetic():
     assert abs(up["achieved"] - 4 * 8192 * 4096 * 14336 / 1e-3 / 1e12) < 1e-9 * up["achieved"]
 
 
+def test_dram_frac():
+    """Measured DRAM bytes per launch over the live time, against the HBM
+    copy peak: 1.7 GB in 0.5 ms is 3.4 TB/s, half of a 6.8 TB/s peak."""
+    assert abs(bench.dram_frac(1.7e9, 0.5, {"hbm_gbs": 6800.0}) - 0.5) < 1e-12
+
+
 def test_launches_per_step():
     from mixture_experts_ffn_token_b200.workloads import WORKLOADS
     W = WORKLOADS
