@@ -341,6 +341,23 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t mask) {
                : "memory");
 }
 
+// ------------------------------------------------ L2 eviction priority
+// A cache policy (createpolicy) under which the lines an access writes are
+// the first candidates for replacement in L2, before lines of normal
+// priority; a later access under the default policy makes them normal again.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 16-byte store under a cache policy.
+__device__ __forceinline__ void st_v4_policy(uint4* ptr, const uint4& v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w), "l"(pol)
+               : "memory");
+}
+
 // --------------------------------------------------------------- numerics
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
