@@ -20,6 +20,10 @@ LAUNCH_FORMS = [
     {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_CTA_PAIR": "2"},
     {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_CTA_PAIR": "2"},
     {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_B_ONE_BOX": "0"},
+    # row f1: the gate_up GEMM gathers its rows of x itself (the gather
+    # kernel still runs where the router weight scales the rows)
+    {"MOE_B200_SINGLE_LAUNCH": "1", "MOE_B200_FUSED_GATHER": "1", "MOE_B200_TILE_SCHEDULE": "static"},
+    {"MOE_B200_SINGLE_LAUNCH": "0", "MOE_B200_FUSED_GATHER": "1"},
 ]
 
 NUM_CASES = 256

@@ -1,7 +1,8 @@
 """A seeded sweep of random small layer configurations (tests/random_configs.py)
 through moe_forward / moe_forward_ex against the fp64 oracle, cycling the
 launch forms: single launch in static and dynamic tile order, two launches,
-CTA pairs in both, four-box B copies. Same bars as every parity test:
+CTA pairs in both, four-box B copies, and the gate_up GEMM gathering its
+own rows (row f1) in one and in two launches. Same bars as every parity test:
 routing bit-exact, router weights 1e-5 relative, output 2e-2 * max|ref|."""
 import pytest
 
