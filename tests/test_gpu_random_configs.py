@@ -4,9 +4,14 @@ launch forms: single launch in static and dynamic tile order, two launches,
 CTA pairs in both, four-box B copies, and the gate_up GEMM gathering its
 own rows (row f1) in one and in two launches. Same bars as every parity test:
 routing bit-exact, router weights 1e-5 relative, output 2e-2 * max|ref|."""
+import numpy as np
 import pytest
+import torch
 
-from gpu_helpers import run_and_check, run_and_check_ex
+import oracle
+from gpu_helpers import LayerRun, run_and_check, run_and_check_ex, to_dev
+from mixture_experts_ffn_token_b200 import abi
+from mixture_experts_ffn_token_b200.workloads import make_inputs
 from random_configs import NUM_CASES, random_workload
 
 pytestmark = pytest.mark.gpu
@@ -21,3 +26,43 @@ def test_random_config(i, monkeypatch):
         run_and_check_ex(wl, seed=i)
     else:
         run_and_check(wl, seed=i)
+
+
+@pytest.mark.parametrize("i", range(0, NUM_CASES, 4))
+def test_random_config_stages(i, monkeypatch):
+    """The staged entry points on every fourth draw (without the extensions,
+    which only moe_forward_ex takes): moe_route -> moe_create_indices (with
+    the inverse) -> moe_grouped_ffn give moe_forward's routing and output bit
+    for bit, and the CSR is the oracle's counting sort."""
+    wl, form = random_workload(i)
+    wl = wl.replace(mask_frac=0.0, weight_first=False, num_shared=0, shared_dim=0)
+    for key, value in form.items():
+        monkeypatch.setenv(key, value)
+    inp = make_inputs(wl, seed=i)
+    d = to_dev(inp)
+    run = LayerRun(wl, d)
+    assert run.status == 0
+    T, k, E, S = wl.num_tokens, wl.top_k, wl.num_experts, wl.num_sink
+    cfg = run.cfg
+    ws = torch.empty_like(run.ws)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    sink = torch.empty((T, S), dtype=torch.float32, device="cuda") if S > 0 else None
+    abi.moe_route(cfg, d["logits"], idx, w, sink_weights=sink, expert_bias=d["expert_bias"],
+                  global_scale=d["global_scale"])
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    abi.moe_create_indices(cfg, idx, off, perm, inv, ws)
+    out = torch.empty((T, wl.hidden_dim), dtype=torch.bfloat16, device="cuda")
+    abi.moe_grouped_ffn(cfg, d["x"], d["W_gu"], d["b_gu"], d["W_d"], d["b_d"], off, perm, w, out, ws)
+    torch.cuda.synchronize()
+    assert abi.moe_device_status(ws) == 0
+    assert torch.equal(idx, run.idx) and torch.equal(w, run.w)
+    if S > 0:
+        assert torch.equal(sink, run.sink)
+    _, o_ref, p_ref, i_ref = oracle.create_indices(idx.cpu().numpy(), E)
+    assert np.array_equal(off.cpu().numpy(), o_ref)
+    assert np.array_equal(perm.cpu().numpy(), p_ref)
+    assert np.array_equal(inv.cpu().numpy(), i_ref)
+    assert torch.equal(out, run.out)
