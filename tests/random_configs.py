@@ -65,3 +65,36 @@ def random_workload(i):
             kw["num_shared"] = r.choice([0, S])  # shared expert i is gated by sink lane i
         kw["shared_dim"] = 8 * r.randint(1, 48) if kw["num_shared"] > 0 else 0
     return WORKLOADS["tiny"].replace(**kw), LAUNCH_FORMS[i % len(LAUNCH_FORMS)]
+
+
+NUM_MIDSIZE = 48
+
+
+def random_midsize_workload(i):
+    """The i-th mid-size draw: a few thousand routed rows, so each launch has
+    hundreds to thousands of tiles over ragged expert segments (several tiles
+    per CTA, every wrap of the tile-number ring, the dynamic counter under
+    contention), at sizes whose oracle over the every-tile token sample
+    still takes seconds. No extensions."""
+    r = random.Random(104729 * (i + 1))
+    router = r.choice(["softmax_topk", "sigmoid_sink"])
+    E = r.choice([4, 8, 16, 40, 64, 128, 160])
+    if router == "sigmoid_sink":
+        lanes = r.choice([4, 8, 16])
+        k = r.randint(1, min(E, lanes, 8))
+        S = lanes - k
+    else:
+        k = r.randint(1, min(E, 8))
+        S = 0
+    T = r.randint(400, max(400, 6000 // k))
+    H = 8 * r.randint(32, 128)
+    D = 8 * r.randint(32, 128)
+    activation = r.choice(["silu", "swigluoai", "gelu_tanh"])
+    kw = dict(name=f"midsize{i}", num_tokens=T, hidden_dim=H, num_experts=E, top_k=k, moe_dim=D, router=router,
+              num_sink=S, gate_up_format=r.choice(["concatenated", "interleaved"]), activation=activation,
+              alpha=1.702 if activation == "swigluoai" else 0.0,
+              limit=0.0 if activation == "gelu_tanh" else r.choice([0.0, 7.0]), has_bias=r.random() < 0.5,
+              logits_kind="normal", logits_std=r.choice([0.5, 1.0, 2.0]),
+              expert_bias_range=0.1 if router == "sigmoid_sink" else 0.0,
+              route_scale=2.5 if router == "sigmoid_sink" else 1.0)
+    return WORKLOADS["tiny"].replace(**kw), LAUNCH_FORMS[i % len(LAUNCH_FORMS)]

@@ -9,10 +9,10 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import LayerRun, run_and_check, run_and_check_ex, to_dev
+from gpu_helpers import LayerRun, every_tile_tokens, oracle_route, run_and_check, run_and_check_ex, to_dev
 from mixture_experts_ffn_token_b200 import abi
 from mixture_experts_ffn_token_b200.workloads import make_inputs
-from random_configs import NUM_CASES, random_workload
+from random_configs import NUM_CASES, NUM_MIDSIZE, random_midsize_workload, random_workload
 
 pytestmark = pytest.mark.gpu
 
@@ -66,3 +66,17 @@ def test_random_config_stages(i, monkeypatch):
     assert np.array_equal(perm.cpu().numpy(), p_ref)
     assert np.array_equal(inv.cpu().numpy(), i_ref)
     assert torch.equal(out, run.out)
+
+
+@pytest.mark.parametrize("i", range(NUM_MIDSIZE))
+def test_random_midsize_every_tile(i, monkeypatch):
+    """Mid-size random draws, the layer output compared on the tokens whose
+    rows reach every 128-row piece of every expert (so every tile of both
+    contractions has rows compared), routing on every token."""
+    wl, form = random_midsize_workload(i)
+    for key, value in form.items():
+        monkeypatch.setenv(key, value)
+    inp = make_inputs(wl, seed=i)
+    idx_ref, _, _ = oracle_route(wl, inp)
+    tokens = every_tile_tokens(idx_ref, wl.num_experts)
+    run_and_check(wl, seed=i, sample_tokens=tokens)
