@@ -10,6 +10,7 @@ broken copies of the oracle, by test_oracle_mutants.py.
 import json
 import math
 import os
+import random
 from decimal import Decimal, getcontext
 
 import numpy as np
@@ -443,6 +444,64 @@ def pin_shared_experts():
     assert torch.allclose(torch.from_numpy(got), ref * torch.from_numpy(gates), rtol=1e-12, atol=1e-12)
 
 
+def pin_random_brute_force():
+    """Seeded random shapes and options, each part against its brute-force
+    form: the FFN (with the router weight first and a token mask on some
+    draws) against the per-token loop of dense torch MLPs, the sink router
+    against the decimal sigma_i / sum sigma_j with a sorted selection, the
+    softmax router on tie-prone logits against a sort by (-z, e) and the
+    renormalised exponentials, the CSR against a sort by (expert, slot)."""
+    r = random.Random(2024)
+    for case in range(150):
+        T, H, E, D = r.randint(1, 8), r.randint(1, 20), r.randint(1, 6), r.randint(1, 10)
+        k = r.randint(1, E)
+        fmt = r.choice(["concatenated", "interleaved"])
+        act = r.choice(["silu", "swigluoai", "gelu_tanh"])
+        alpha = ALPHA if act == "swigluoai" else 0.0
+        limit = 0.0 if act == "gelu_tanh" else r.choice([0.0, 0.3, LIMIT])
+        L = rand_layer(T=T, H=H, E=E, k=k, D=D, seed=1000 + case, bias=r.random() < 0.5)
+        weight_first = r.random() < 0.3
+        mask = np.array([r.random() < 0.7 for _ in range(T)], np.uint8) if r.random() < 0.3 else None
+        got = oracle.expert_ffn(L["xb"], L["idx"].numpy(), L["w"].numpy(), L["Wgub"], L["Wdb"], L["bgub"], L["bdb"],
+                                fmt, act, alpha, limit, weight_first=weight_first, token_mask=mask)
+        ref = (brute_force_weight_first if weight_first else brute_force_layer)(L, act, fmt, alpha, limit)
+        if mask is not None:
+            ref[torch.from_numpy(mask == 0)] = 0.0        # a masked token's row is zero
+        assert torch.allclose(torch.from_numpy(got), ref, rtol=1e-12, atol=1e-12), (case, fmt, act, limit)
+    g = torch.Generator().manual_seed(2025)
+    for case in range(60):
+        E, S = r.randint(1, 40), r.randint(0, 4)
+        k = r.randint(1, E)
+        scale, gscale = r.choice([0.5, 1.0, 2.5]), r.choice([1.0, 0.7])
+        zt = (torch.randn(6, E + S, generator=g) * r.choice([0.5, 2.0, 6.0])).numpy()
+        bias = (torch.rand(E, generator=g) * 0.2 - 0.1).numpy() if r.random() < 0.7 else None
+        idx, w, sw = oracle.route_sigmoid_sink(zt, E, S, k, bias, scale, gscale)
+        sig = (1.0 / (1.0 + np.exp(-zt[:, :E].astype(np.float64)))).astype(np.float32)
+        score = sig + (0 if bias is None else bias)
+        for t in range(6):
+            assert idx[t].tolist() == sorted(range(E), key=lambda e: (-float(score[t, e]), e))[:k], (case, t)
+            ref = d_sink_weights_logspace([float(zt[t, e]) for e in idx[t]] + [float(v) for v in zt[t, E:]],
+                                          scale * gscale)
+            got = list(w[t]) + list(sw[t])
+            assert all(close(a, b, 1e-12, 1e-300) for a, b in zip(got, ref)), (case, t, got, ref)
+        # softmax top-k on logits with frequent ties (few distinct values):
+        # descending, ties to the lowest index, softmax over the selected
+        zt = torch.randint(-3, 4, (6, E), generator=g).float().numpy() * r.choice([0.5, 1.0])
+        idx, w = oracle.route_softmax_topk(zt, E, k)
+        for t in range(6):
+            sel = sorted(range(E), key=lambda e: (-float(zt[t, e]), e))[:k]
+            assert idx[t].tolist() == sel, (case, t)
+            ex = np.exp(zt[t, sel].astype(np.float64) - zt[t, sel].max())
+            assert np.allclose(w[t], ex / ex.sum(), rtol=1e-14, atol=0), (case, t)
+        T = r.randint(1, 60)
+        idx = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32).numpy()
+        counts, offsets, perm, inv = oracle.create_indices(idx, E)
+        flat = idx.reshape(-1)
+        assert perm.tolist() == sorted(range(flat.size), key=lambda s: (flat[s], s))
+        assert offsets.tolist() == [0] + np.cumsum(np.bincount(flat, minlength=E)).tolist()
+        assert (inv[perm] == np.arange(flat.size)).all()
+
+
 ALL_PINS = [pin_activation_closed_forms, pin_activation_library_routines, pin_softmax_router, pin_sink_router,
             pin_csr, pin_ffn_dense_reduction, pin_ffn_brute_force, pin_ffn_invariants, pin_ffn_empty_experts,
-            pin_weight_first, pin_token_mask, pin_shared_experts]
+            pin_weight_first, pin_token_mask, pin_shared_experts, pin_random_brute_force]
