@@ -38,6 +38,21 @@ MUTANTS = {
     "weight_first_also_weights_output": ("const double wj = weight_first ? 1.0 : w[t * k + j];",
                                          "const double wj = w[t * k + j];"),
     "mask_ignored": ("      if (token_mask && token_mask[t] == 0) continue;\n", ""),
+    "sink_global_scale_dropped": ("double scale = route_scale * global_scale;", "double scale = route_scale;"),
+    "sink_lanes_read_from_column_zero": ("log_sigmoid(logit_at(logits, logits_is_bf16, t, stride, E + i))",
+                                         "log_sigmoid(logit_at(logits, logits_is_bf16, t, stride, i))"),
+    "silu_applied_to_up": ("return g / (1.0 + std::exp(-g)) * u;", "return u / (1.0 + std::exp(-u)) * g;"),
+    "gelu_drops_one_half": ("return 0.5 * g * (1.0 + std::tanh(inner)) * u;", "return g * (1.0 + std::tanh(inner)) * u;"),
+    "silu_gate_clamped_from_below": ("g = std::min(g, limit);\n        u = std::min(std::max(u, -limit), limit);\n      }\n      return g / (1.0",
+                                     "g = std::min(std::max(g, -limit), limit);\n        u = std::min(std::max(u, -limit), limit);\n      }\n      return g / (1.0"),
+    "down_bias_dropped": ("ys[c] = b_d ? bf16_bits_to_double(b_d[static_cast<int64_t>(e) * H + c]) : 0.0;", "ys[c] = 0.0;"),
+    "csr_inverse_off_by_one": ("if (inv) inv[s] = pos;", "if (inv) inv[s] = pos + 1;"),
+    "softmax_weights_not_normalised": ("w[t * k + j] = std::exp(z[idx[t * k + j]] - m) / sum;",
+                                       "w[t * k + j] = std::exp(z[idx[t * k + j]] - m);"),
+    "interleaved_up_is_gate": ("double u = gate_up_format == 0 ? a[D + i] : a[2 * i + 1];",
+                               "double u = gate_up_format == 0 ? a[D + i] : a[2 * i];"),
+    "concatenated_up_is_gate": ("double u = gate_up_format == 0 ? a[D + i] : a[2 * i + 1];",
+                                "double u = gate_up_format == 0 ? a[i] : a[2 * i + 1];"),
 }
 
 
