@@ -12,7 +12,13 @@ namespace moe {
 //   MOE_B200_PDL_COOP=0        none on the two cooperative launches (CSR build, FFN)
 //   MOE_B200_CSR_FUSED=0       the CSR build as three launches
 //   MOE_B200_SINGLE_LAUNCH=0   the two grouped GEMMs as two launches
-//   MOE_B200_CTA_PAIR=2        CTA-pair GEMM tiles (two launches)
+//   MOE_B200_CTA_PAIR=2        CTA-pair GEMM tiles (single launch unless
+//                              MOE_B200_SINGLE_LAUNCH=0)
+//   MOE_B200_PAIR_COOP=0       the single-launch pair without the cooperative
+//                              attribute (its grid still comes from the
+//                              cluster occupancy query; if some cluster is not
+//                              resident, the bounded dependency waits report
+//                              a timeout instead of hanging)
 //   MOE_B200_B_ONE_BOX=0       four copies per B stage tile
 //   MOE_B200_TILE_SCHEDULE=static|dynamic   tile order of the single launch
 //   MOE_B200_FUSED_GATHER=1    the gate_up GEMM gathers its rows of x itself
