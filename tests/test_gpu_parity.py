@@ -137,13 +137,34 @@ def test_programmatic_launch_changes_nothing(name, monkeypatch):
     wl = SMALL[name]
     d = to_dev(make_inputs(wl, 13))
     outs = []
-    for pdl in ("1", "0"):
+    # every launch programmatic; none; every launch but the two cooperative
+    # ones (CSR build, FFN)
+    for pdl, coop in (("1", "1"), ("0", "1"), ("1", "0")):
         monkeypatch.setenv("MOE_B200_PDL", pdl)
+        monkeypatch.setenv("MOE_B200_PDL_COOP", coop)
         run = LayerRun(wl, d)
         assert run.status == 0
         outs.append((run.out.clone(), run.idx.clone(), run.w.clone()))
-    for a, b in zip(outs[0], outs[1]):
-        assert torch.equal(a, b)
+    for other in outs[1:]:
+        for a, b in zip(outs[0], other):
+            assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name", ["sink_small", "mixtral_small"])
+def test_single_launch_pair_without_cooperative_attribute(name, monkeypatch):
+    """MOE_B200_PAIR_COOP=0: the single-launch CTA-pair FFN as a plain
+    clustered launch, its grid sized by the cluster occupancy query, gives
+    the cooperative launch's bits (on an idle GPU every cluster is resident)."""
+    wl = SMALL[name]
+    d = to_dev(make_inputs(wl, 14))
+    set_variant(monkeypatch, "single_launch_cta_pair")
+    outs = []
+    for coop in ("1", "0"):
+        monkeypatch.setenv("MOE_B200_PAIR_COOP", coop)
+        run = LayerRun(wl, d)
+        assert run.status == 0, f"device status {run.status:#x}"
+        outs.append(run.out.clone())
+    assert torch.equal(outs[0], outs[1])
 
 
 @pytest.mark.parametrize("name", sorted(ALIGNED))
