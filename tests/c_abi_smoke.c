@@ -5,6 +5,12 @@
  *     bit for bit, and two moe_forward calls agree,
  *   - the device status word is clean,
  *   - the output is finite and not all zero.
+ *   - moe_forward_timed, and moe_forward_ex without extensions, give
+ *     moe_forward's bits; moe_forward_ex with a token mask zeroes the masked
+ *     rows and leaves every other row's bits unchanged;
+ *   - moe_single_launch_ffn answers 0 or 1, moe_workspace_size_ex(NULL)
+ *     equals moe_workspace_size, and moe_create_indices_noalloc builds the
+ *     same CSR as moe_create_indices.
  * Prints "ok" and exits 0 on success; the GPU test suite compiles and runs it. */
 #include <cuda_runtime.h>
 #include <math.h>
@@ -147,6 +153,106 @@ int main(void) {
   if (memcmp(h1, h2, (size_t)T * H * 2) != 0) {
     fprintf(stderr, "two moe_forward calls differ\n");
     return 1;
+  }
+
+  /* whether the two GEMMs run as one launch: a status and a 0/1 answer */
+  int32_t single = -1;
+  CHECK_MOE(moe_single_launch_ffn(&single));
+  if (single != 0 && single != 1) {
+    fprintf(stderr, "moe_single_launch_ffn gave %d\n", single);
+    return 1;
+  }
+
+  /* moe_forward_timed: the same bits, and every stage interval non-negative */
+  {
+    cudaEvent_t ev[MOE_NUM_STAGE_EVENTS];
+    for (int i = 0; i < MOE_NUM_STAGE_EVENTS; ++i) CHECK_CUDA(cudaEventCreate(&ev[i]));
+    CHECK_MOE(moe_forward_timed(&cfg, x, logits, NULL, NULL, wgu, NULL, wd, NULL, out2, NULL, NULL, NULL, ws,
+                                ws_bytes, 0, (void* const*)ev));
+    CHECK_CUDA(cudaDeviceSynchronize());
+    for (int i = 0; i + 1 < MOE_NUM_STAGE_EVENTS; ++i) {
+      float ms = -1.0f;
+      CHECK_CUDA(cudaEventElapsedTime(&ms, ev[i], ev[i + 1]));
+      if (!(ms >= 0.0f)) {
+        fprintf(stderr, "stage %d interval %f\n", i, ms);
+        return 1;
+      }
+    }
+    for (int i = 0; i < MOE_NUM_STAGE_EVENTS; ++i) CHECK_CUDA(cudaEventDestroy(ev[i]));
+    CHECK_CUDA(cudaMemcpy(h2, out2, (size_t)T * H * 2, cudaMemcpyDeviceToHost));
+    if (memcmp(h1, h2, (size_t)T * H * 2) != 0) {
+      fprintf(stderr, "moe_forward_timed differs from moe_forward\n");
+      return 1;
+    }
+  }
+
+  /* moe_forward_ex: no extensions gives moe_forward's bits; a token mask
+     zeroes the masked rows and leaves every other row's bits unchanged */
+  {
+    size_t ws_ex = 0;
+    CHECK_MOE(moe_workspace_size_ex(&cfg, NULL, &ws_ex));
+    if (ws_ex != ws_bytes) {
+      fprintf(stderr, "moe_workspace_size_ex(NULL) %zu != moe_workspace_size %zu\n", ws_ex, ws_bytes);
+      return 1;
+    }
+    CHECK_MOE(moe_forward_ex(&cfg, NULL, x, logits, NULL, NULL, wgu, NULL, wd, NULL, out2, NULL, NULL, NULL, ws,
+                             ws_bytes, 0, NULL));
+    CHECK_CUDA(cudaDeviceSynchronize());
+    CHECK_CUDA(cudaMemcpy(h2, out2, (size_t)T * H * 2, cudaMemcpyDeviceToHost));
+    if (memcmp(h1, h2, (size_t)T * H * 2) != 0) {
+      fprintf(stderr, "moe_forward_ex without extensions differs from moe_forward\n");
+      return 1;
+    }
+    uint8_t hmask[T];
+    for (int t = 0; t < T; ++t) hmask[t] = (uint8_t)(t % 3 != 1);
+    uint8_t* mask;
+    CHECK_CUDA(cudaMalloc((void**)&mask, (size_t)T));
+    CHECK_CUDA(cudaMemcpy(mask, hmask, (size_t)T, cudaMemcpyHostToDevice));
+    moe_extras_t ex;
+    memset(&ex, 0, sizeof(ex));
+    ex.token_mask = mask;
+    CHECK_MOE(moe_workspace_size_ex(&cfg, &ex, &ws_ex));
+    void* ws2;
+    CHECK_CUDA(cudaMalloc(&ws2, ws_ex));
+    CHECK_MOE(moe_forward_ex(&cfg, &ex, x, logits, NULL, NULL, wgu, NULL, wd, NULL, out2, NULL, NULL, NULL, ws2,
+                             ws_ex, 0, NULL));
+    CHECK_CUDA(cudaDeviceSynchronize());
+    CHECK_CUDA(cudaMemcpy(h2, out2, (size_t)T * H * 2, cudaMemcpyDeviceToHost));
+    for (int t = 0; t < T; ++t) {
+      const int same = memcmp(h1 + (size_t)t * H, h2 + (size_t)t * H, (size_t)H * 2) == 0;
+      int zero = 1;
+      for (int c = 0; c < H; ++c) zero &= from_bf16(h2[(size_t)t * H + c]) == 0.0f;
+      if (hmask[t] ? !same : !zero) {
+        fprintf(stderr, "token %d: masked rows must be zero, the others unchanged\n", t);
+        return 1;
+      }
+    }
+    CHECK_CUDA(cudaFree(ws2));
+    CHECK_CUDA(cudaFree(mask));
+  }
+
+  /* moe_create_indices_noalloc: the same CSR without a workspace */
+  {
+    int32_t *off2, *perm2;
+    CHECK_CUDA(cudaMalloc((void**)&off2, (size_t)(E + 1) * 4));
+    CHECK_CUDA(cudaMalloc((void**)&perm2, (size_t)T * k * 4));
+    CHECK_MOE(moe_create_indices_noalloc(&cfg, idx, off2, perm2, NULL, 0));
+    CHECK_CUDA(cudaDeviceSynchronize());
+    int32_t a[E + 1], b[E + 1];
+    int32_t* pa = (int32_t*)malloc((size_t)T * k * 4);
+    int32_t* pb = (int32_t*)malloc((size_t)T * k * 4);
+    CHECK_CUDA(cudaMemcpy(a, offsets, (size_t)(E + 1) * 4, cudaMemcpyDeviceToHost));
+    CHECK_CUDA(cudaMemcpy(b, off2, (size_t)(E + 1) * 4, cudaMemcpyDeviceToHost));
+    CHECK_CUDA(cudaMemcpy(pa, perm, (size_t)T * k * 4, cudaMemcpyDeviceToHost));
+    CHECK_CUDA(cudaMemcpy(pb, perm2, (size_t)T * k * 4, cudaMemcpyDeviceToHost));
+    if (memcmp(a, b, sizeof(a)) != 0 || memcmp(pa, pb, (size_t)T * k * 4) != 0) {
+      fprintf(stderr, "moe_create_indices_noalloc differs from moe_create_indices\n");
+      return 1;
+    }
+    free(pa);
+    free(pb);
+    CHECK_CUDA(cudaFree(off2));
+    CHECK_CUDA(cudaFree(perm2));
   }
 
   double sum = 0.0;
